@@ -1,0 +1,180 @@
+/*
+ * kdv.h -- C ABI of the B200 (sm_100a) tree-verify MLA attention library.
+ *
+ * What the library computes. In a speculative-decoding verify step, every
+ * node of a draft tree is evaluated in parallel; each node attends over the
+ * KV cache under a visibility mask that follows the tree, in a fused
+ * multi-head latent attention that absorbs the latent projection (page "The
+ * Architecture of Diagnosis", section "Phase 1: Custom CUDA Kernels", item 2).
+ * A latent KV row is c_kv[kv_lora_rank=512] || k_rope[qk_rope_head_dim=64],
+ * 576 elements per token per layer (page "From Diagnosis to Deployment",
+ * section "The Second Thread"). The KV cache is paged with page_size=1
+ * (page "The Architecture of Diagnosis", section "The Discrepancy That
+ * Revealed the Truth", item 2). A long prefix and the tree tail can be
+ * evaluated separately and merged (page "The Three Acts of Engineering",
+ * reference [1]); the merge is a log-sum-exp combine.
+ *
+ * Definitions used by every call (T = tree size, L = prefix length, H heads):
+ *   Anc*(t) = {t, parent[t], parent[parent[t]], ...}       (self included)
+ *   visible keys of node t: prefix keys 0..L-1 and tree keys L+u, u in Anc*(t)
+ *   s[t,h,j] = scale * (q_lat[t,h] . c_kv[j] + q_rope[t,h] . k_rope[j])
+ *   o_lat[t,h] = sum_j softmax_j(s) c_kv[j],  lse[t,h] = ln sum_j exp(s[t,h,j])
+ *
+ * Conventions.
+ *   - Every call returns a kdv_status; 0 (KDV_OK) is success. No exceptions.
+ *   - Array arguments are DEVICE pointers owned by the caller unless marked
+ *     HOST. The library allocates no device memory: scratch space is the
+ *     caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Host-side argument checks run before any launch and
+ *     return KDV_ERR_INVALID_ARG / KDV_ERR_UNSUPPORTED without touching the GPU.
+ *   - Bad data that only the device can see (a parent[] entry out of range,
+ *     a page-table slot >= num_slots, a device length that disagrees with the
+ *     host copy) is reported through the optional int32 `d_err` flag (0 = ok,
+ *     otherwise the first KDV_DERR_* code seen). The offending access is
+ *     skipped and the kernel finishes normally; nothing traps.
+ *   - Rows are node-major: global row = (tree_off[b] + t) * H + h.
+ */
+#ifndef KDV_H_
+#define KDV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDV_API __attribute__((visibility("default")))
+#else
+#define KDV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDV_OK = 0,
+  KDV_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad size or stride     */
+  KDV_ERR_UNSUPPORTED = -2, /* valid but not implemented (dims, T > 64, batch) */
+  KDV_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required     */
+  KDV_ERR_CUDA = -4         /* a CUDA launch or runtime call failed           */
+} kdv_status;
+
+/* Codes written to *d_err by kernels (first error wins). */
+#define KDV_DERR_BAD_PARENT 1  /* parent[i] not in {-1} U [0, i)            */
+#define KDV_DERR_BAD_SLOT 2    /* page_table entry outside [0, num_slots)   */
+#define KDV_DERR_BAD_LENGTH 3  /* device prefix_len differs from host copy  */
+#define KDV_DERR_BAD_TOKEN 4   /* tree-accept: token id out of range        */
+
+/* Element type of q and kv. */
+#define KDV_BF16 0
+#define KDV_F32 1
+
+/* Kernel family for kdv_verify_attn. AUTO picks the tensor-core kernel when
+ * its shape constraints hold (bf16, d_latent=512, d_rope=64), else SIMT. */
+#define KDV_IMPL_AUTO 0
+#define KDV_IMPL_SIMT 1
+#define KDV_IMPL_TC 2
+
+#define KDV_MAX_TREE 64    /* nodes per tree (one 64-bit mask word)          */
+#define KDV_MAX_BATCH 128  /* requests per kdv_verify_attn call              */
+
+/* Human-readable name of a status code (static string, never NULL). */
+KDV_API const char* kdv_status_string(kdv_status s);
+
+/* Library ABI version (major*100 + minor). */
+KDV_API int32_t kdv_version(void);
+
+/*
+ * kdv_tree_mask_build -- parent[] to ancestor bitmask (bit-exact).
+ * The tree visibility mask of page "The Architecture of Diagnosis", section
+ * "Phase 1: Custom CUDA Kernels", item 2: bit u of mask[i] is set iff node u
+ * is node i itself or one of its ancestors.
+ *   parent   [sumT] int32, per-request local indices; parent[i] in {-1} U [0,i)
+ *            (-1 marks a root; several roots form a forest)
+ *   tree_off [batch+1] int32 CSR offsets into parent/mask, or NULL for a single
+ *            request of max_T nodes (batch must then be 1)
+ *   batch    >= 1;  max_T in [1, 64], an upper bound on every request's T
+ *   mask     [sumT] uint64 out
+ *   depth    [sumT] int32 out, nullable: edges to the root (root = 0)
+ *   d_err    nullable; KDV_DERR_BAD_PARENT for a malformed parent[] (that
+ *            node's mask is written as 0)
+ */
+KDV_API kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
+                               int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
+                               void* stream);
+
+/*
+ * Parameters of kdv_verify_attn (absorbed-form tree-verify attention).
+ *
+ * Key addressing: logical key j of request b (0 <= j < L_b + T_b) is pool row
+ *   page_table[kv_off[b] + j]   when page_table != NULL (page_size = 1), or
+ *   kv_off[b] + j               when page_table == NULL (contiguous).
+ * Key L_b + u holds tree node u's own latent row (written by the caller).
+ *
+ * Splits: with S splits, split s of request b covers the logical keys
+ *   [s*c_b, min((s+1)*c_b, L_b+T_b)),  c_b = 64 * ceil((L_b+T_b) / (64*S)),
+ * so a split may be empty (o = 0, lse = -inf). num_splits = 0 lets the
+ * library choose S per request to fill the GPU and merge the partials in the
+ * workspace; num_splits >= 1 forces S for every request.
+ */
+typedef struct kdv_verify_params {
+  int32_t batch;         /* B in [1, KDV_MAX_BATCH]                              */
+  int32_t num_heads;     /* H >= 1                                               */
+  int32_t d_latent;      /* D_c: 512 for the TC kernel; 1..512 for SIMT          */
+  int32_t d_rope;        /* D_r: 64 for the TC kernel; 0..64 for SIMT            */
+  float scale;           /* softmax scale on q.k (e.g. 1/sqrt(d_nope + d_rope))  */
+  int32_t dtype;         /* KDV_BF16 or KDV_F32 (q and kv)                       */
+  int32_t impl;          /* KDV_IMPL_AUTO / _SIMT / _TC                          */
+  const void* q;         /* [sumT*H][q_row_stride], row = q_lat || q_rope        */
+  int64_t q_row_stride;  /* elements between q rows; 0 means D_c + D_r           */
+  const void* kv;        /* pool [num_slots][D_c + D_r], row = c_kv || k_rope    */
+  int64_t num_slots;     /* rows in the pool                                     */
+  const int32_t* page_table;   /* [kv_off[B]] slots, or NULL (contiguous)        */
+  const int32_t* kv_off;       /* [B+1] device                                   */
+  const int32_t* tree_off;     /* [B+1] device                                   */
+  const int32_t* prefix_len;   /* [B] device, nullable: checked against host     */
+  const int32_t* h_prefix_len; /* [B] HOST copy of L_b (used to plan the grid)   */
+  const int32_t* h_tree_T;     /* [B] HOST copy of T_b in [1, 64]                */
+  const uint64_t* mask;        /* [sumT] from kdv_tree_mask_build                */
+  int32_t num_splits;          /* 0 = auto, >= 1 forced                          */
+  int32_t return_partials;     /* 1: write o_part/lse_part, no merge (S forced)  */
+  float* o;              /* [sumT*H][D_c] out (unused when return_partials)      */
+  float* lse;            /* [sumT*H] out, nullable                               */
+  float* o_part;         /* [S][sumT*H][D_c] out when return_partials            */
+  float* lse_part;       /* [S][sumT*H] out when return_partials                 */
+  void* workspace;       /* caller-owned scratch, >= kdv_verify_attn_workspace   */
+  size_t workspace_bytes;
+  int32_t* d_err;        /* nullable device error flag                           */
+} kdv_verify_params;
+
+/* Bytes of workspace kdv_verify_attn needs for these parameters (the plan
+ * depends only on the host fields). Writes *bytes; may be 0. */
+KDV_API kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t* bytes);
+
+/*
+ * kdv_verify_attn -- tree-verify MLA attention in absorbed form.
+ * Absorbed Q.K^T over D_c + D_r dims, online softmax, P.V over the D_c latent
+ * dims (V is the c_kv part of the same pool row), optional per-split LSE and
+ * the split merge. Output o_lat is fp32 [sumT*H][D_c]; lse is the natural-log
+ * log-sum-exp of the scaled logits. Requirements: q, kv 16-byte aligned;
+ * q_row_stride*elem and (D_c+D_r)*elem multiples of 16 bytes for the TC kernel.
+ */
+KDV_API kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream);
+
+/*
+ * kdv_combine -- log-sum-exp merge of S split partials (the prefix / tree-tail
+ * merge of page "The Three Acts of Engineering", reference [1]):
+ *   LSE = ln sum_k exp(lse_k),  o = sum_k exp(lse_k - LSE) o_k.
+ * A part with lse_k = -inf weighs nothing; a row whose parts are all empty
+ * gets o = 0 and LSE = -inf.
+ *   o_part [S][rows][d] fp32, lse_part [S][rows] fp32, o [rows][d], lse [rows]
+ *   (lse nullable). S >= 1, rows >= 0, d >= 1.
+ */
+KDV_API kdv_status kdv_combine(const float* o_part, const float* lse_part, int32_t S, int64_t rows,
+                       int32_t d, float* o, float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDV_H_ */

@@ -1,0 +1,263 @@
+// kdv_api.cu -- the C ABI: argument checks, split planning, launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "kdv_internal.cuh"
+
+using namespace kdv;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+bool tc_shape_ok(const kdv_verify_params* p) {
+  return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64;
+}
+
+int resolve_impl(const kdv_verify_params* p) {
+  if (p->impl == KDV_IMPL_SIMT || p->impl == KDV_IMPL_TC) return p->impl;
+  return tc_shape_ok(p) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
+}
+
+// Host-side checks that need no device access.
+kdv_status check_params(const kdv_verify_params* p, int impl) {
+  if (p == nullptr) return KDV_ERR_INVALID_ARG;
+  if (p->batch < 1) return KDV_ERR_INVALID_ARG;
+  if (p->batch > KDV_MAX_BATCH) return KDV_ERR_UNSUPPORTED;
+  if (p->num_heads < 1) return KDV_ERR_INVALID_ARG;
+  if (p->dtype != KDV_BF16 && p->dtype != KDV_F32) return KDV_ERR_INVALID_ARG;
+  if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC) return KDV_ERR_INVALID_ARG;
+  if (p->d_latent < 1 || p->d_rope < 0) return KDV_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return KDV_ERR_INVALID_ARG;
+  if (p->h_prefix_len == nullptr || p->h_tree_T == nullptr) return KDV_ERR_INVALID_ARG;
+  for (int b = 0; b < p->batch; ++b) {
+    if (p->h_prefix_len[b] < 0) return KDV_ERR_INVALID_ARG;
+    if (p->h_tree_T[b] < 1) return KDV_ERR_INVALID_ARG;
+    if (p->h_tree_T[b] > KDV_MAX_TREE) return KDV_ERR_UNSUPPORTED;
+  }
+  if (p->num_splits < 0) return KDV_ERR_INVALID_ARG;
+  if (p->return_partials != 0 && p->return_partials != 1) return KDV_ERR_INVALID_ARG;
+  if (p->return_partials && p->num_splits < 1) return KDV_ERR_INVALID_ARG;
+  if (impl == KDV_IMPL_TC) {
+    if (!tc_shape_ok(p)) return KDV_ERR_UNSUPPORTED;
+  } else {
+    if (p->d_latent > 512 || p->d_rope > 64) return KDV_ERR_UNSUPPORTED;
+  }
+  return KDV_OK;
+}
+
+kdv_status check_pointers(const kdv_verify_params* p, int impl) {
+  const int64_t D_q = (int64_t)p->d_latent + p->d_rope;
+  const int64_t stride = p->q_row_stride == 0 ? D_q : p->q_row_stride;
+  if (stride < D_q) return KDV_ERR_INVALID_ARG;
+  if (!p->q || !p->kv || !p->kv_off || !p->tree_off || !p->mask) return KDV_ERR_INVALID_ARG;
+  if (p->num_slots < 0) return KDV_ERR_INVALID_ARG;
+  if (p->return_partials) {
+    if (!p->o_part || !p->lse_part) return KDV_ERR_INVALID_ARG;
+  } else if (!p->o) {
+    return KDV_ERR_INVALID_ARG;
+  }
+  const size_t esz = p->dtype == KDV_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(p->q) % esz) || (reinterpret_cast<uintptr_t>(p->kv) % esz))
+    return KDV_ERR_INVALID_ARG;
+  if (impl == KDV_IMPL_TC) {
+    // TMA needs 16-byte aligned bases and row pitches
+    if (!aligned16(p->q) || !aligned16(p->kv)) return KDV_ERR_INVALID_ARG;
+    if ((stride * (int64_t)esz) % 16 != 0) return KDV_ERR_INVALID_ARG;
+  }
+  float* outs[4] = {p->o, p->lse, p->o_part, p->lse_part};
+  for (float* f : outs)
+    if (f && (reinterpret_cast<uintptr_t>(f) & 3u)) return KDV_ERR_INVALID_ARG;
+  return KDV_OK;
+}
+
+// Build the grid / split plan. Fills *ws_bytes with the workspace needed.
+kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, size_t* ws_bytes) {
+  std::memset(plan, 0, sizeof(*plan));
+  const int B = p->batch, H = p->num_heads;
+  const int rows_per_tile = impl == KDV_IMPL_TC ? TC_ROWS : SIMT_ROWS;
+  plan->B = B;
+  plan->H = H;
+  plan->rows_per_tile = rows_per_tile;
+  int64_t tree_acc = 0;
+  double work = 0.0;
+  for (int b = 0; b < B; ++b) {
+    plan->L[b] = p->h_prefix_len[b];
+    plan->T[b] = p->h_tree_T[b];
+    plan->tree_base[b] = (int32_t)tree_acc;
+    tree_acc += p->h_tree_T[b];
+    const int64_t rows_b = (int64_t)p->h_tree_T[b] * H;
+    const int64_t tiles = (rows_b + rows_per_tile - 1) / rows_per_tile;
+    if (tiles > INT_MAX / 2 || rows_b > INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
+    plan->tiles[b] = (int32_t)tiles;
+    work += (double)tiles * ((double)p->h_prefix_len[b] + p->h_tree_T[b]);
+  }
+  if (tree_acc * (int64_t)H > INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
+  plan->total_rows = (int32_t)(tree_acc * H);
+
+  // splits per request
+  const int sms = device_sm_count();
+  // TC: one item is a 2-CTA cluster, so sms/2 items fill the GPU once.
+  // SIMT: 8-warp CTAs, several per SM.
+  const double target_items = impl == KDV_IMPL_TC ? sms / 2 : 4.0 * sms;
+  const int min_keys = impl == KDV_IMPL_TC ? 4 * TC_KEYS : 128;
+  for (int b = 0; b < B; ++b) {
+    const int64_t n_b = (int64_t)plan->L[b] + plan->T[b];
+    int64_t S;
+    if (p->num_splits >= 1) {
+      S = p->num_splits;
+    } else {
+      const double per_item = work / target_items;          // keys x tiles per item
+      S = (int64_t)std::floor((double)n_b * plan->tiles[b] / std::max(per_item, 1.0) / plan->tiles[b]);
+      S = std::max<int64_t>(1, std::min<int64_t>(S, (n_b + min_keys - 1) / min_keys));
+    }
+    if (S > 4096) return KDV_ERR_UNSUPPORTED;
+    const int64_t chunk = TC_KEYS * ((n_b + TC_KEYS * S - 1) / (TC_KEYS * S));
+    plan->S[b] = (int32_t)S;
+    plan->chunk[b] = (int32_t)std::max<int64_t>(chunk, TC_KEYS);
+  }
+  int64_t items = 0, parts = 0;
+  bool all_one = true;
+  for (int b = 0; b < B; ++b) {
+    plan->item_base[b] = (int32_t)items;
+    items += (int64_t)plan->tiles[b] * plan->S[b];
+    plan->part_base[b] = (int32_t)parts;
+    parts += (int64_t)plan->S[b] * plan->T[b] * H;
+    if (plan->S[b] != 1) all_one = false;
+    if (items > INT_MAX / 4 || parts > INT_MAX / 4) return KDV_ERR_UNSUPPORTED;
+  }
+  plan->item_base[B] = (int32_t)items;
+  plan->n_items = (int32_t)items;
+  *ws_bytes = 0;
+  if (p->return_partials) {
+    plan->out_mode = OUT_PARTIALS;
+  } else if (all_one) {
+    plan->out_mode = OUT_DIRECT;
+  } else {
+    plan->out_mode = OUT_WORKSPACE;
+    const size_t o_bytes = (size_t)parts * p->d_latent * sizeof(float);
+    const size_t o_al = (o_bytes + 255) & ~(size_t)255;
+    *ws_bytes = o_al + (size_t)parts * sizeof(float);
+  }
+  return KDV_OK;
+}
+
+kdv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KDV_OK : KDV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kdv_status_string(kdv_status s) {
+  switch (s) {
+    case KDV_OK: return "KDV_OK";
+    case KDV_ERR_INVALID_ARG: return "KDV_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+    case KDV_ERR_UNSUPPORTED: return "KDV_ERR_UNSUPPORTED: valid request the library does not implement";
+    case KDV_ERR_WORKSPACE: return "KDV_ERR_WORKSPACE: workspace missing or too small";
+    case KDV_ERR_CUDA: return "KDV_ERR_CUDA: a CUDA launch or runtime call failed";
+  }
+  return "KDV_ERR_UNKNOWN";
+}
+
+int32_t kdv_version(void) { return 100; }
+
+kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
+                               int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
+                               void* stream) {
+  if (parent == nullptr || mask == nullptr) return KDV_ERR_INVALID_ARG;
+  if (batch < 1 || max_T < 1) return KDV_ERR_INVALID_ARG;
+  if (max_T > KDV_MAX_TREE) return KDV_ERR_UNSUPPORTED;
+  if (tree_off == nullptr && batch != 1) return KDV_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(mask) & 7u) return KDV_ERR_INVALID_ARG;
+  return cuda_status(launch_mask_build(parent, tree_off, batch, max_T, mask, depth, d_err,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t* bytes) {
+  if (p == nullptr || bytes == nullptr) return KDV_ERR_INVALID_ARG;
+  const int impl = resolve_impl(p);
+  kdv_status st = check_params(p, impl);
+  if (st != KDV_OK) return st;
+  VerifyPlan plan;
+  return make_plan(p, impl, &plan, bytes);
+}
+
+kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
+  if (p == nullptr) return KDV_ERR_INVALID_ARG;
+  const int impl = resolve_impl(p);
+  kdv_status st = check_params(p, impl);
+  if (st != KDV_OK) return st;
+  st = check_pointers(p, impl);
+  if (st != KDV_OK) return st;
+  VerifyPlan plan;
+  size_t need = 0;
+  st = make_plan(p, impl, &plan, &need);
+  if (st != KDV_OK) return st;
+  if (need > 0) {
+    if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace))
+      return KDV_ERR_WORKSPACE;
+  }
+  VerifyArgs a;
+  a.q = p->q;
+  a.q_row_stride = p->q_row_stride == 0 ? (int64_t)p->d_latent + p->d_rope : p->q_row_stride;
+  a.kv = p->kv;
+  a.num_slots = p->num_slots;
+  a.page_table = p->page_table;
+  a.kv_off = p->kv_off;
+  a.tree_off = p->tree_off;
+  a.prefix_len = p->prefix_len;
+  a.mask = p->mask;
+  a.D_c = p->d_latent;
+  a.D_r = p->d_rope;
+  a.scale = p->scale;
+  a.d_err = p->d_err;
+  float* ws_o = nullptr;
+  float* ws_l = nullptr;
+  if (plan.out_mode == OUT_DIRECT) {
+    a.o = p->o;
+    a.lse = p->lse;
+  } else if (plan.out_mode == OUT_PARTIALS) {
+    a.o = p->o_part;
+    a.lse = p->lse_part;
+  } else {
+    const size_t parts = (size_t)plan.part_base[plan.B - 1] +
+                         (size_t)plan.S[plan.B - 1] * plan.T[plan.B - 1] * plan.H;
+    const size_t o_bytes = parts * p->d_latent * sizeof(float);
+    ws_o = static_cast<float*>(p->workspace);
+    ws_l = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + ((o_bytes + 255) & ~(size_t)255));
+    a.o = ws_o;
+    a.lse = ws_l;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = impl == KDV_IMPL_TC ? launch_verify_tc(a, plan, s)
+                                      : launch_verify_simt(a, plan, p->dtype, s);
+  if (e != cudaSuccess) return KDV_ERR_CUDA;
+  if (plan.out_mode == OUT_WORKSPACE)
+    e = launch_combine_plan(ws_o, ws_l, plan, p->d_latent, p->o, p->lse, s);
+  return cuda_status(e);
+}
+
+kdv_status kdv_combine(const float* o_part, const float* lse_part, int32_t S, int64_t rows,
+                       int32_t d, float* o, float* lse, void* stream) {
+  if (S < 1 || rows < 0 || d < 1) return KDV_ERR_INVALID_ARG;
+  if (rows > 0 && (o_part == nullptr || lse_part == nullptr || o == nullptr))
+    return KDV_ERR_INVALID_ARG;
+  return cuda_status(launch_combine_uniform(o_part, lse_part, S, rows, d, o, lse,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// kdv_internal.cuh -- shared declarations of the CUDA library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kdv.h"
+
+namespace kdv {
+
+// Split / grid plan computed on the host from the HOST length copies and
+// passed to kernels by value (kernel parameters, ~5 KB). Work item i of the
+// grid maps to request b with item_base[b] <= i < item_base[b+1]; inside the
+// request, local = i - item_base[b] = split * tiles[b] + row_tile, so items
+// that run side by side share one split's keys in L2.
+struct VerifyPlan {
+  int32_t B;
+  int32_t H;
+  int32_t n_items;
+  int32_t rows_per_tile;
+  int32_t out_mode;        // OUT_DIRECT / OUT_PARTIALS / OUT_WORKSPACE
+  int32_t total_rows;      // sumT * H
+  int32_t item_base[KDV_MAX_BATCH + 1];
+  int32_t L[KDV_MAX_BATCH];
+  int32_t T[KDV_MAX_BATCH];
+  int32_t S[KDV_MAX_BATCH];
+  int32_t chunk[KDV_MAX_BATCH];
+  int32_t tiles[KDV_MAX_BATCH];
+  int32_t tree_base[KDV_MAX_BATCH];   // tree_off[b] (from the host T copies)
+  int32_t part_base[KDV_MAX_BATCH];   // first workspace partial row of request b
+};
+
+enum OutMode : int32_t { OUT_DIRECT = 0, OUT_PARTIALS = 1, OUT_WORKSPACE = 2 };
+
+// Everything a verify kernel reads or writes besides the plan.
+struct VerifyArgs {
+  const void* q;
+  int64_t q_row_stride;
+  const void* kv;
+  int64_t num_slots;
+  const int32_t* page_table;
+  const int32_t* kv_off;
+  const int32_t* tree_off;
+  const int32_t* prefix_len;
+  const uint64_t* mask;
+  int32_t D_c;
+  int32_t D_r;
+  float scale;
+  float* o;          // OUT_DIRECT: [rows][D_c]; OUT_PARTIALS: [S][rows][D_c]; OUT_WORKSPACE: ws
+  float* lse;        // matching lse array (may be null in OUT_DIRECT)
+  int32_t* d_err;
+};
+
+// Where the (request b, split s, local row r) result goes, in rows of D_c.
+__host__ __device__ inline int64_t out_row_index(const VerifyPlan& p, int b, int s, int r) {
+  const int64_t row_global = (int64_t)p.tree_base[b] * p.H + r;
+  if (p.out_mode == OUT_DIRECT) return row_global;
+  if (p.out_mode == OUT_PARTIALS) return (int64_t)s * p.total_rows + row_global;
+  return (int64_t)p.part_base[b] + (int64_t)s * ((int64_t)p.T[b] * p.H) + r;
+}
+
+__device__ inline void record_error(int32_t* d_err, int32_t code) {
+  if (d_err != nullptr) atomicCAS(d_err, 0, code);
+}
+
+// Find the request of work item `item` (B <= 128: a short scan).
+__device__ inline int plan_request(const VerifyPlan& p, int item) {
+  int b = 0;
+  while (b + 1 < p.B && p.item_base[b + 1] <= item) ++b;
+  return b;
+}
+
+// Launchers (each returns cudaGetLastError() of its launch).
+cudaError_t launch_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
+                              int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
+                              cudaStream_t stream);
+cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t dtype,
+                               cudaStream_t stream);
+cudaError_t launch_verify_tc(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
+cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, int32_t S,
+                                   int64_t rows, int32_t d, float* o, float* lse,
+                                   cudaStream_t stream);
+cudaError_t launch_combine_plan(const float* ws_o, const float* ws_lse, const VerifyPlan& p,
+                                int32_t d, float* o, float* lse, cudaStream_t stream);
+
+// TC kernel tile geometry (shared with the planner).
+constexpr int TC_ROWS = 128;   // query rows per CTA pair
+constexpr int TC_KEYS = 64;    // keys per pipeline stage
+constexpr int SIMT_ROWS = 8;   // query rows per SIMT CTA (one warp per row)
+
+}  // namespace kdv

@@ -1,0 +1,255 @@
+"""Thin Python binding of the C-ABI library ``libkdv.so`` (include/kdv.h).
+
+Argument marshalling only: each ``kdv_*`` function here takes torch tensors
+(device memory, allocated by the caller) and host lists, passes raw pointers
+and sizes to the C entry point of the same name, and raises ``KdvError`` on a
+non-zero status. Every step of the computation runs in the library's CUDA
+kernels. There is no fallback: if ``libkdv.so`` is missing, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkdv.so")
+
+KDV_OK = 0
+KDV_ERR_INVALID_ARG = -1
+KDV_ERR_UNSUPPORTED = -2
+KDV_ERR_WORKSPACE = -3
+KDV_ERR_CUDA = -4
+
+KDV_DERR_BAD_PARENT = 1
+KDV_DERR_BAD_SLOT = 2
+KDV_DERR_BAD_LENGTH = 3
+KDV_DERR_BAD_TOKEN = 4
+
+KDV_BF16 = 0
+KDV_F32 = 1
+KDV_IMPL_AUTO = 0
+KDV_IMPL_SIMT = 1
+KDV_IMPL_TC = 2
+KDV_MAX_TREE = 64
+KDV_MAX_BATCH = 128
+
+# Every entry point include/kdv.h declares (checked by the CPU tests).
+EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
+            "kdv_verify_attn_workspace", "kdv_verify_attn", "kdv_combine")
+
+
+class KdvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class VerifyParams(ctypes.Structure):
+    """Mirror of ``kdv_verify_params`` (field order and types must match kdv.h)."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+        ("d_latent", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("dtype", ctypes.c_int32), ("impl", ctypes.c_int32),
+        ("q", ctypes.c_void_p), ("q_row_stride", ctypes.c_int64),
+        ("kv", ctypes.c_void_p), ("num_slots", ctypes.c_int64),
+        ("page_table", ctypes.c_void_p), ("kv_off", ctypes.c_void_p),
+        ("tree_off", ctypes.c_void_p), ("prefix_len", ctypes.c_void_p),
+        ("h_prefix_len", ctypes.POINTER(ctypes.c_int32)),
+        ("h_tree_T", ctypes.POINTER(ctypes.c_int32)),
+        ("mask", ctypes.c_void_p), ("num_splits", ctypes.c_int32),
+        ("return_partials", ctypes.c_int32),
+        ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("o_part", ctypes.c_void_p), ("lse_part", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("d_err", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libkdv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                               "or speculative_tree_verify_mla_b200/build.py")
+        lib = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        lib.kdv_status_string.argtypes = [c.c_int]
+        lib.kdv_status_string.restype = c.c_char_p
+        lib.kdv_version.argtypes = []
+        lib.kdv_version.restype = c.c_int32
+        lib.kdv_tree_mask_build.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int32,
+                                            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
+        lib.kdv_tree_mask_build.restype = c.c_int
+        lib.kdv_verify_attn_workspace.argtypes = [c.POINTER(VerifyParams), c.POINTER(c.c_size_t)]
+        lib.kdv_verify_attn_workspace.restype = c.c_int
+        lib.kdv_verify_attn.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
+        lib.kdv_verify_attn.restype = c.c_int
+        lib.kdv_combine.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int64, c.c_int32,
+                                    c.c_void_p, c.c_void_p, c.c_void_p]
+        lib.kdv_combine.restype = c.c_int
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().kdv_status_string(int(status)).decode()
+
+
+def kdv_version() -> int:
+    return int(load().kdv_version())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        if torch.cuda.is_available():
+            return int(torch.cuda.current_stream().cuda_stream) or None
+        return None
+    if isinstance(stream, torch.cuda.Stream):
+        return int(stream.cuda_stream) or None
+    return int(stream) or None
+
+
+def _check(status: int, where: str):
+    if status != KDV_OK:
+        raise KdvError(status, where)
+
+
+def kdv_tree_mask_build(parent: torch.Tensor, tree_off: Optional[torch.Tensor], batch: int,
+                        max_T: int, mask: torch.Tensor, depth: Optional[torch.Tensor] = None,
+                        d_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """parent[] -> ancestor bitmask (int64 tensor holding the uint64 bits)."""
+    _check(load().kdv_tree_mask_build(_ptr(parent), _ptr(tree_off), int(batch), int(max_T),
+                                      _ptr(mask), _ptr(depth), _ptr(d_err), _stream(stream)),
+           "kdv_tree_mask_build")
+
+
+def make_params(**kw) -> VerifyParams:
+    """Build a VerifyParams from keyword arguments (tensors become pointers)."""
+    p = VerifyParams()
+    keep = []
+    for k, v in kw.items():
+        if k in ("h_prefix_len", "h_tree_T"):
+            arr = (ctypes.c_int32 * len(v))(*[int(x) for x in v])
+            keep.append(arr)
+            setattr(p, k, ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)))
+        elif isinstance(v, torch.Tensor):
+            setattr(p, k, int(v.data_ptr()))
+        elif v is None:
+            setattr(p, k, None)
+        else:
+            setattr(p, k, v)
+    p._keep = keep          # keep host arrays alive with the struct
+    return p
+
+
+def kdv_verify_attn_workspace(params: VerifyParams) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().kdv_verify_attn_workspace(ctypes.byref(params), ctypes.byref(n)),
+           "kdv_verify_attn_workspace")
+    return int(n.value)
+
+
+def kdv_verify_attn(params: VerifyParams, stream=None) -> None:
+    _check(load().kdv_verify_attn(ctypes.byref(params), _stream(stream)), "kdv_verify_attn")
+
+
+def kdv_combine(o_part: torch.Tensor, lse_part: torch.Tensor, S: int, rows: int, d: int,
+                o: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(load().kdv_combine(_ptr(o_part), _ptr(lse_part), int(S), int(rows), int(d), _ptr(o),
+                              _ptr(lse), _stream(stream)), "kdv_combine")
+
+
+# ---------------------------------------------------------------------------
+# Device-resident problem (upload once, call many times).
+# ---------------------------------------------------------------------------
+class DeviceCase:
+    """A ``datagen.VerifyCase`` uploaded to the GPU, plus output buffers.
+
+    ``run()`` calls kdv_tree_mask_build then kdv_verify_attn through the C ABI.
+    """
+
+    def __init__(self, case, device="cuda", impl: int = KDV_IMPL_AUTO, num_splits: int = 0,
+                 return_partials: bool = False):
+        dev = torch.device(device)
+        self.case = case
+        self.impl = impl
+        self.num_splits = num_splits
+        self.return_partials = return_partials
+        tdt = torch.bfloat16 if case.dtype == "bf16" else torch.float32
+        self.dtype = KDV_BF16 if case.dtype == "bf16" else KDV_F32
+        self.q = torch.from_numpy(case.q).to(tdt).to(dev)
+        self.kv = torch.from_numpy(case.kv).to(tdt).to(dev)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        self.parent = i32(case.parent)
+        self.tree_off = i32(case.tree_off)
+        self.kv_off = i32(case.kv_off)
+        self.prefix_len = i32(case.prefix_len)
+        self.page_table = i32(case.page_table) if case.page_table is not None else None
+        sumT = int(case.tree_off[-1])
+        self.mask = torch.zeros(sumT, dtype=torch.int64, device=dev)
+        self.depth = torch.zeros(sumT, dtype=torch.int32, device=dev)
+        self.d_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        rows = case.rows
+        self.o = torch.empty(rows, case.D_c, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(rows, dtype=torch.float32, device=dev)
+        S = max(1, num_splits)
+        self.o_part = self.lse_part = None
+        if return_partials:
+            self.o_part = torch.empty(S, rows, case.D_c, dtype=torch.float32, device=dev)
+            self.lse_part = torch.empty(S, rows, dtype=torch.float32, device=dev)
+        self.params = self._params()
+        self.ws_bytes = kdv_verify_attn_workspace(self.params)
+        self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.params.workspace = int(self.workspace.data_ptr())
+        self.params.workspace_bytes = self.ws_bytes
+
+    def _params(self) -> VerifyParams:
+        c = self.case
+        return make_params(
+            batch=c.batch, num_heads=c.H, d_latent=c.D_c, d_rope=c.D_r, scale=c.scale,
+            dtype=self.dtype, impl=self.impl, q=self.q, q_row_stride=c.D_q, kv=self.kv,
+            num_slots=int(c.kv.shape[0]), page_table=self.page_table, kv_off=self.kv_off,
+            tree_off=self.tree_off, prefix_len=self.prefix_len,
+            h_prefix_len=[int(x) for x in c.prefix_len], h_tree_T=[int(x) for x in c.tree_T],
+            mask=self.mask, num_splits=self.num_splits,
+            return_partials=1 if self.return_partials else 0, o=self.o, lse=self.lse,
+            o_part=self.o_part, lse_part=self.lse_part, workspace=None, workspace_bytes=0,
+            d_err=self.d_err)
+
+    def build_mask(self, stream=None):
+        c = self.case
+        kdv_tree_mask_build(self.parent, self.tree_off, c.batch, int(max(c.tree_T)), self.mask,
+                            self.depth, self.d_err, stream)
+
+    def verify(self, stream=None):
+        kdv_verify_attn(self.params, stream)
+
+    def run(self, stream=None):
+        self.build_mask(stream)
+        self.verify(stream)
+        return self
+
+    def results(self):
+        """(o, lse) or (o_part, lse_part) as numpy arrays, after a sync."""
+        torch.cuda.synchronize()
+        if self.return_partials:
+            return self.o_part.cpu().numpy(), self.lse_part.cpu().numpy()
+        return self.o.cpu().numpy(), self.lse.cpu().numpy()
+
+    def error_flag(self) -> int:
+        torch.cuda.synchronize()
+        return int(self.d_err.item())

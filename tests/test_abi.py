@@ -1,0 +1,142 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared entry
+point, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from speculative_tree_verify_mla_b200 import build, kdv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kdv.load()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"KDV_API[^;(]*?\b(kdv_\w+)\s*\(", txt))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert names == set(kdv.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in (0, -1, -2, -3, -4):
+        assert kdv.status_string(s).startswith("KDV_")
+    assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
+    assert kdv.kdv_version() == 100
+
+
+def test_params_struct_layout(tmp_path):
+    """ctypes mirror matches the C struct: compile a probe against kdv.h."""
+    fields = [f[0] for f in kdv.VerifyParams._fields_]
+    src = tmp_path / "probe.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "kdv.h"\nint main(void){'
+                   + "".join(f'printf("%zu\\n", offsetof(kdv_verify_params, {f}));' for f in fields)
+                   + 'printf("%zu\\n", sizeof(kdv_verify_params)); return 0;}')
+    exe = tmp_path / "probe"
+    import subprocess
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    want = [getattr(kdv.VerifyParams, f).offset for f in fields] + [ctypes.sizeof(kdv.VerifyParams)]
+    assert got == want
+
+
+def _params(**over):
+    base = dict(batch=1, num_heads=4, d_latent=64, d_rope=16, scale=0.1, dtype=kdv.KDV_F32,
+                impl=kdv.KDV_IMPL_SIMT, q=None, q_row_stride=0, kv=None, num_slots=10,
+                page_table=None, kv_off=None, tree_off=None, prefix_len=None,
+                h_prefix_len=[5], h_tree_T=[3], mask=None, num_splits=0, return_partials=0,
+                o=None, lse=None, o_part=None, lse_part=None, workspace=None,
+                workspace_bytes=0, d_err=None)
+    base.update(over)
+    return kdv.make_params(**base)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(batch=0), kdv.KDV_ERR_INVALID_ARG),
+    (dict(batch=129, h_prefix_len=[1] * 129, h_tree_T=[1] * 129), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(num_heads=0), kdv.KDV_ERR_INVALID_ARG),
+    (dict(h_tree_T=[65]), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(h_tree_T=[0]), kdv.KDV_ERR_INVALID_ARG),
+    (dict(h_prefix_len=[-1]), kdv.KDV_ERR_INVALID_ARG),
+    (dict(dtype=7), kdv.KDV_ERR_INVALID_ARG),
+    (dict(impl=kdv.KDV_IMPL_TC), kdv.KDV_ERR_UNSUPPORTED),          # f32, 64/16 dims
+    (dict(d_latent=513), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(d_rope=65), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(num_splits=-1), kdv.KDV_ERR_INVALID_ARG),
+    (dict(return_partials=1, num_splits=0), kdv.KDV_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), kdv.KDV_ERR_INVALID_ARG),
+])
+def test_host_validation(lib, over, status):
+    p = _params(**over)
+    n = ctypes.c_size_t(0)
+    assert lib.kdv_verify_attn_workspace(ctypes.byref(p), ctypes.byref(n)) == status
+    assert lib.kdv_verify_attn(ctypes.byref(p), None) == status
+
+
+def test_null_pointers_rejected_before_launch(lib):
+    p = _params()
+    assert lib.kdv_verify_attn(ctypes.byref(p), None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_tc_alignment_rejected(lib):
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
+                q=0x1002, kv=0x2000, kv_off=0x3000, tree_off=0x4000, mask=0x5000, o=0x6000)
+    assert lib.kdv_verify_attn(ctypes.byref(p), None) == kdv.KDV_ERR_INVALID_ARG
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
+                q=0x1000, kv=0x2000, kv_off=0x3000, tree_off=0x4000, mask=0x5000, o=0x6000,
+                q_row_stride=577)
+    assert lib.kdv_verify_attn(ctypes.byref(p), None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(lib):
+    # forced single split: direct output, no workspace
+    assert kdv.kdv_verify_attn_workspace(_params(num_splits=1)) == 0
+    # forced 3 splits, merged by the library: 3 * T*H partial rows of (D_c + 1) floats
+    n = kdv.kdv_verify_attn_workspace(_params(num_splits=3))
+    parts = 3 * 3 * 4
+    assert n == ((parts * 64 * 4 + 255) // 256) * 256 + parts * 4
+    # partials returned to the caller: no workspace
+    assert kdv.kdv_verify_attn_workspace(_params(num_splits=3, return_partials=1)) == 0
+
+
+def test_mask_build_validation(lib):
+    f = lib.kdv_tree_mask_build
+    assert f(None, None, 1, 4, 0x1000, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(0x1000, None, 1, 65, 0x2000, None, None, None) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(0x1000, None, 2, 4, 0x2000, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(0x1000, None, 1, 0, 0x2000, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(0x1000, None, 1, 4, 0x2004, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_combine_validation(lib):
+    f = lib.kdv_combine
+    assert f(None, None, 0, 4, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(None, None, 2, 4, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(None, None, 2, -1, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_library_has_no_oracle_dependency():
+    """The CUDA library and its binding never reference the oracle."""
+    pkg = os.path.join(ROOT, "speculative_tree_verify_mla_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, fn
+                assert "kdv_oracle" not in txt, fn
