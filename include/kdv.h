@@ -64,6 +64,8 @@ typedef enum {
 #define KDV_DERR_BAD_SLOT 2    /* page_table entry outside [0, num_slots)   */
 #define KDV_DERR_BAD_LENGTH 3  /* device prefix_len differs from host copy  */
 #define KDV_DERR_BAD_TOKEN 4   /* tree-accept: token id out of range        */
+#define KDV_DERR_TIMEOUT 5     /* a bounded in-kernel wait ran out (~1 s);
+                                  the kernel stopped early, output invalid  */
 
 /* Element type of q and kv. */
 #define KDV_BF16 0

@@ -30,7 +30,7 @@ bool tc_shape_ok(const kdv_verify_params* p) {
 
 int resolve_impl(const kdv_verify_params* p) {
   if (p->impl == KDV_IMPL_SIMT || p->impl == KDV_IMPL_TC) return p->impl;
-  return tc_shape_ok(p) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
+  return (tc_shape_ok(p) && p->page_table == nullptr) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
 }
 
 // Host-side checks that need no device access.
@@ -54,6 +54,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->return_partials && p->num_splits < 1) return KDV_ERR_INVALID_ARG;
   if (impl == KDV_IMPL_TC) {
     if (!tc_shape_ok(p)) return KDV_ERR_UNSUPPORTED;
+    if (p->page_table != nullptr) return KDV_ERR_UNSUPPORTED;
   } else {
     if (p->d_latent > 512 || p->d_rope > 64) return KDV_ERR_UNSUPPORTED;
   }

@@ -28,6 +28,7 @@ KDV_DERR_BAD_PARENT = 1
 KDV_DERR_BAD_SLOT = 2
 KDV_DERR_BAD_LENGTH = 3
 KDV_DERR_BAD_TOKEN = 4
+KDV_DERR_TIMEOUT = 5
 
 KDV_BF16 = 0
 KDV_F32 = 1
