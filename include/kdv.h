@@ -114,7 +114,7 @@ KDV_API kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tre
  * Key L_b + u holds tree node u's own latent row (written by the caller).
  *
  * Splits: with S splits, split s of request b covers the logical keys
- *   [s*c_b, min((s+1)*c_b, L_b+T_b)),  c_b = 64 * ceil((L_b+T_b) / (64*S)),
+ *   [s*c_b, min((s+1)*c_b, L_b+T_b)),  c_b = 128 * ceil((L_b+T_b) / (128*S)),
  * so a split may be empty (o = 0, lse = -inf). num_splits = 0 lets the
  * library choose S per request to fill the GPU and merge the partials in the
  * workspace; num_splits >= 1 forces S for every request.
@@ -152,6 +152,14 @@ typedef struct kdv_verify_params {
 /* Bytes of workspace kdv_verify_attn needs for these parameters (the plan
  * depends only on the host fields). Writes *bytes; may be 0. */
 KDV_API kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t* bytes);
+
+/* The plan kdv_verify_attn would use for these parameters (host fields only):
+ * splits[b] = S for request b (length batch, nullable) and *grid_items = the
+ * number of work items (2-CTA clusters for the TC kernel, CTAs for SIMT),
+ * nullable. Lets a caller size o_part for return_partials with the automatic
+ * split count. */
+KDV_API kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* splits,
+                                        int32_t* grid_items);
 
 /*
  * kdv_verify_attn -- tree-verify MLA attention in absorbed form.

@@ -115,7 +115,7 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   // TC: one item is a 2-CTA cluster, so sms/2 items fill the GPU once.
   // SIMT: 8-warp CTAs, several per SM.
   const double target_items = impl == KDV_IMPL_TC ? sms / 2 : 4.0 * sms;
-  const int min_keys = impl == KDV_IMPL_TC ? 4 * TC_KEYS : 128;
+  const int min_keys = impl == KDV_IMPL_TC ? 2 * TC_KEYS : 128;
   for (int b = 0; b < B; ++b) {
     const int64_t n_b = (int64_t)plan->L[b] + plan->T[b];
     int64_t S;
@@ -127,9 +127,9 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
       S = std::max<int64_t>(1, std::min<int64_t>(S, (n_b + min_keys - 1) / min_keys));
     }
     if (S > 4096) return KDV_ERR_UNSUPPORTED;
-    const int64_t chunk = TC_KEYS * ((n_b + TC_KEYS * S - 1) / (TC_KEYS * S));
+    const int64_t chunk = SPLIT_ALIGN * ((n_b + SPLIT_ALIGN * S - 1) / (SPLIT_ALIGN * S));
     plan->S[b] = (int32_t)S;
-    plan->chunk[b] = (int32_t)std::max<int64_t>(chunk, TC_KEYS);
+    plan->chunk[b] = (int32_t)std::max<int64_t>(chunk, SPLIT_ALIGN);
   }
   int64_t items = 0, parts = 0;
   bool all_one = true;
@@ -195,6 +195,21 @@ kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t* bytes) 
   if (st != KDV_OK) return st;
   VerifyPlan plan;
   return make_plan(p, impl, &plan, bytes);
+}
+
+kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* splits, int32_t* grid_items) {
+  if (p == nullptr) return KDV_ERR_INVALID_ARG;
+  const int impl = resolve_impl(p);
+  kdv_status st = check_params(p, impl);
+  if (st != KDV_OK) return st;
+  VerifyPlan plan;
+  size_t bytes = 0;
+  st = make_plan(p, impl, &plan, &bytes);
+  if (st != KDV_OK) return st;
+  if (splits)
+    for (int b = 0; b < plan.B; ++b) splits[b] = plan.S[b];
+  if (grid_items) *grid_items = plan.n_items;
+  return KDV_OK;
 }
 
 kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {

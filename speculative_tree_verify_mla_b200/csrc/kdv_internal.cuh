@@ -85,7 +85,8 @@ cudaError_t launch_combine_plan(const float* ws_o, const float* ws_lse, const Ve
 
 // TC kernel tile geometry (shared with the planner).
 constexpr int TC_ROWS = 128;   // query rows per CTA pair
-constexpr int TC_KEYS = 64;    // keys per pipeline stage
+constexpr int TC_KEYS = 128;   // keys per S / P tile of the tensor-core kernel
+constexpr int SPLIT_ALIGN = 128;  // split boundaries are multiples of this many keys
 constexpr int SIMT_ROWS = 8;   // query rows per SIMT CTA (one warp per row)
 
 }  // namespace kdv

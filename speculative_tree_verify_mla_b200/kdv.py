@@ -40,7 +40,8 @@ KDV_MAX_BATCH = 128
 
 # Every entry point include/kdv.h declares (checked by the CPU tests).
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
-            "kdv_verify_attn_workspace", "kdv_verify_attn", "kdv_combine")
+            "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
+            "kdv_combine")
 
 
 class KdvError(RuntimeError):
@@ -91,6 +92,8 @@ def load() -> ctypes.CDLL:
         lib.kdv_tree_mask_build.restype = c.c_int
         lib.kdv_verify_attn_workspace.argtypes = [c.POINTER(VerifyParams), c.POINTER(c.c_size_t)]
         lib.kdv_verify_attn_workspace.restype = c.c_int
+        lib.kdv_verify_attn_plan.argtypes = [c.POINTER(VerifyParams), c.c_void_p, c.c_void_p]
+        lib.kdv_verify_attn_plan.restype = c.c_int
         lib.kdv_verify_attn.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
         lib.kdv_verify_attn.restype = c.c_int
         lib.kdv_combine.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int64, c.c_int32,
@@ -162,6 +165,15 @@ def kdv_verify_attn_workspace(params: VerifyParams) -> int:
     _check(load().kdv_verify_attn_workspace(ctypes.byref(params), ctypes.byref(n)),
            "kdv_verify_attn_workspace")
     return int(n.value)
+
+
+def kdv_verify_attn_plan(params: VerifyParams):
+    """(splits per request, grid work items) that kdv_verify_attn would use."""
+    splits = (ctypes.c_int32 * max(1, params.batch))()
+    items = ctypes.c_int32(0)
+    _check(load().kdv_verify_attn_plan(ctypes.byref(params), splits, ctypes.byref(items)),
+           "kdv_verify_attn_plan")
+    return [int(splits[i]) for i in range(params.batch)], int(items.value)
 
 
 def kdv_verify_attn(params: VerifyParams, stream=None) -> None:

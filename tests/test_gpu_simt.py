@@ -92,7 +92,7 @@ def test_partials_and_combine_simt():
     dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_SIMT, num_splits=S, return_partials=True).run()
     o_part, lse_part = dc.results()
     n = 150 + 11
-    c = 64 * math.ceil(n / (64 * S))
+    c = 128 * math.ceil(n / (128 * S))
     for s in range(S):
         lo, hi = min(s * c, n), min((s + 1) * c, n)
         ro, rl = oracle.verify_request(H=3, L=150, parent=case.parent, D_c=48, D_r=16,

@@ -44,7 +44,7 @@ def test_tc_partials_match_oracle_ranges():
     S = 4
     o_part, lse_part = _run(case, splits=S, partials=True)
     n = 300 + 9
-    c = 64 * math.ceil(n / (64 * S))
+    c = 128 * math.ceil(n / (128 * S))
     for s in range(S):
         lo, hi = min(s * c, n), min((s + 1) * c, n)
         if hi <= lo:
