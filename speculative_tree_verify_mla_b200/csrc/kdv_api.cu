@@ -28,8 +28,10 @@ bool tc_shape_ok(const kdv_verify_params* p) {
   return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64;
 }
 
+bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_1SM; }
+
 int resolve_impl(const kdv_verify_params* p) {
-  if (p->impl == KDV_IMPL_SIMT || p->impl == KDV_IMPL_TC) return p->impl;
+  if (p->impl == KDV_IMPL_SIMT || is_tc(p->impl)) return p->impl;
   return (tc_shape_ok(p) && p->page_table == nullptr) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
 }
 
@@ -40,7 +42,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->batch > KDV_MAX_BATCH) return KDV_ERR_UNSUPPORTED;
   if (p->num_heads < 1) return KDV_ERR_INVALID_ARG;
   if (p->dtype != KDV_BF16 && p->dtype != KDV_F32) return KDV_ERR_INVALID_ARG;
-  if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC) return KDV_ERR_INVALID_ARG;
+  if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC_1SM) return KDV_ERR_INVALID_ARG;
   if (p->d_latent < 1 || p->d_rope < 0) return KDV_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return KDV_ERR_INVALID_ARG;
   if (p->h_prefix_len == nullptr || p->h_tree_T == nullptr) return KDV_ERR_INVALID_ARG;
@@ -52,7 +54,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->num_splits < 0) return KDV_ERR_INVALID_ARG;
   if (p->return_partials != 0 && p->return_partials != 1) return KDV_ERR_INVALID_ARG;
   if (p->return_partials && p->num_splits < 1) return KDV_ERR_INVALID_ARG;
-  if (impl == KDV_IMPL_TC) {
+  if (is_tc(impl)) {
     if (!tc_shape_ok(p)) return KDV_ERR_UNSUPPORTED;
     if (p->page_table != nullptr) return KDV_ERR_UNSUPPORTED;
   } else {
@@ -75,7 +77,7 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
   const size_t esz = p->dtype == KDV_BF16 ? 2 : 4;
   if ((reinterpret_cast<uintptr_t>(p->q) % esz) || (reinterpret_cast<uintptr_t>(p->kv) % esz))
     return KDV_ERR_INVALID_ARG;
-  if (impl == KDV_IMPL_TC) {
+  if (is_tc(impl)) {
     // TMA needs 16-byte aligned bases and row pitches
     if (!aligned16(p->q) || !aligned16(p->kv)) return KDV_ERR_INVALID_ARG;
     if ((stride * (int64_t)esz) % 16 != 0) return KDV_ERR_INVALID_ARG;
@@ -90,7 +92,7 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
 kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, size_t* ws_bytes) {
   std::memset(plan, 0, sizeof(*plan));
   const int B = p->batch, H = p->num_heads;
-  const int rows_per_tile = impl == KDV_IMPL_TC ? TC_ROWS : SIMT_ROWS;
+  const int rows_per_tile = impl == KDV_IMPL_TC ? TC2_ROWS : impl == KDV_IMPL_TC_1SM ? TC_ROWS : SIMT_ROWS;
   plan->B = B;
   plan->H = H;
   plan->rows_per_tile = rows_per_tile;
@@ -112,10 +114,18 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
 
   // splits per request
   const int sms = device_sm_count();
-  // TC: one item is a 2-CTA cluster, so sms/2 items fill the GPU once.
-  // SIMT: 8-warp CTAs, several per SM.
-  const double target_items = impl == KDV_IMPL_TC ? sms / 2 : 4.0 * sms;
-  const int min_keys = impl == KDV_IMPL_TC ? 2 * TC_KEYS : 128;
+  // TC: one item is a 4-CTA (TC_1SM: 2-CTA) cluster; clusters only fit within
+  // a GPC, so one wave is what the occupancy query reports (fallback: the SM
+  // count divided by the cluster size). SIMT: 8-warp CTAs, several per SM.
+  double target_items = 4.0 * sms;
+  if (impl == KDV_IMPL_TC) {
+    const int n = tc2_max_active_clusters();
+    target_items = n > 0 ? n : sms / 4;
+  } else if (impl == KDV_IMPL_TC_1SM) {
+    const int n = tc1_max_active_clusters();
+    target_items = n > 0 ? n : sms / 2;
+  }
+  const int min_keys = is_tc(impl) ? 2 * TC_KEYS : 128;
   for (int b = 0; b < B; ++b) {
     const int64_t n_b = (int64_t)plan->L[b] + plan->T[b];
     int64_t S;
@@ -259,8 +269,9 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.lse = ws_l;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = impl == KDV_IMPL_TC ? launch_verify_tc(a, plan, s)
-                                      : launch_verify_simt(a, plan, p->dtype, s);
+  cudaError_t e = impl == KDV_IMPL_TC       ? launch_verify_tc2(a, plan, s)
+                  : impl == KDV_IMPL_TC_1SM ? launch_verify_tc(a, plan, s)
+                                            : launch_verify_simt(a, plan, p->dtype, s);
   if (e != cudaSuccess) return KDV_ERR_CUDA;
   if (plan.out_mode == OUT_WORKSPACE)
     e = launch_combine_plan(ws_o, ws_l, plan, p->d_latent, p->o, p->lse, s);

@@ -77,6 +77,11 @@ cudaError_t launch_mask_build(const int32_t* parent, const int32_t* tree_off, in
 cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t dtype,
                                cudaStream_t stream);
 cudaError_t launch_verify_tc(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
+cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
+// Work items (clusters) of each TC kernel that fit on the device at once,
+// i.e. one wave; 0 when the query fails (no device).
+int tc1_max_active_clusters();
+int tc2_max_active_clusters();
 cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, int32_t S,
                                    int64_t rows, int32_t d, float* o, float* lse,
                                    cudaStream_t stream);
@@ -84,7 +89,8 @@ cudaError_t launch_combine_plan(const float* ws_o, const float* ws_lse, const Ve
                                 int32_t d, float* o, float* lse, cudaStream_t stream);
 
 // TC kernel tile geometry (shared with the planner).
-constexpr int TC_ROWS = 128;   // query rows per CTA pair
+constexpr int TC_ROWS = 128;   // query rows per work item of the 1-SM-MMA kernel
+constexpr int TC2_ROWS = 256;  // query rows per work item of the 2-SM-MMA kernel
 constexpr int TC_KEYS = 128;   // keys per S / P tile of the tensor-core kernel
 constexpr int SPLIT_ALIGN = 128;  // split boundaries are multiples of this many keys
 constexpr int SIMT_ROWS = 8;   // query rows per SIMT CTA (one warp per row)

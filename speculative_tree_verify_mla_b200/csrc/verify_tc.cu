@@ -18,7 +18,8 @@
 //
 //   CTA 0 ("S side"): q_lat (128 x 512 bf16) lives in TMEM (256 columns) and
 //     q_rope (128 x 64) in shared memory; KV arrives by TMA as 16 KB blocks
-//     (128 keys x 64 dims, 128B-swizzled) through a 12-block ring; S = Q K^T
+//     (128 keys x 64 dims, 128B-swizzled), three blocks per barrier, through a
+//     4-stage ring (one wait per 48 KB, not per block); S = Q K^T
 //     (M=128, N=128, K=576) accumulates in one of two 128-column TMEM
 //     buffers. Four softmax warps (one query row per thread) read S, apply the
 //     tree mask, keep the running max and sum, and push P (bf16, 128 x 128, in
@@ -56,8 +57,12 @@ constexpr int QBLOCK_BYTES = ROWS * 128;            // 128 rows x 64 dims
 constexpr int QK_BLOCKS = DQ / 64;                  // 9 (8 latent + 1 rope)
 constexpr int QLAT_BLOCKS = 8;
 constexpr int PV_BLOCKS = DC / 64;                  // 8
-constexpr int KV_SLOTS = 12;                        // S-side ring of 16 KB blocks
-constexpr int KV_FIRST = QLAT_BLOCKS;               // ring position of the first KV block
+constexpr int STAGE_BLOCKS = 3;                     // 16 KB blocks per S-side ring stage
+constexpr int KV_STAGES = 4;                        // S-side ring: 4 stages x 48 KB
+constexpr int KV_SLOTS = KV_STAGES * STAGE_BLOCKS;  // 16 KB block slots in the ring
+constexpr int Q_STAGES = 3;                         // stages holding q_lat at start-up
+constexpr int STAGES_PER_TILE = QK_BLOCKS / STAGE_BLOCKS;
+static_assert(QK_BLOCKS % STAGE_BLOCKS == 0 && QLAT_BLOCKS <= Q_STAGES * STAGE_BLOCKS, "stage geometry");
 constexpr int V_STAGES = 4;
 constexpr int NP = 2;                               // P slots in flight
 constexpr int V_STAGE_BYTES = PV_BLOCKS * VBLOCK_BYTES;  // 32768
@@ -78,7 +83,8 @@ constexpr uint64_t TIMEOUT_NS = 1000000000ull;
 // Shared-memory layout, offsets from a 1024-byte aligned base. Both CTAs use
 // the same offsets so that mapa() addresses of one side line up with the
 // other side's buffers.
-//   S side: [0, 196608) KV ring (12 x 16 KB; slots 0-7 hold q_lat at start-up),
+//   S side: [0, 196608) KV ring (4 stages x 3 blocks of 16 KB; q_lat occupies
+//           the first 8 blocks at start-up),
 //           [196608, 212992) q_rope.
 //   O side: [0, 131072) V ring (4 x 32 KB); P slots; final stats.
 constexpr int OFF_RING = 0;
@@ -98,7 +104,7 @@ static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of shared memory");
 // Barrier slots. Each CTA initialises only its own side's slots; remote
 // arrivals / completions land at the same slot offsets in the other CTA.
 // S side
-constexpr int B_KV_FULL = 0, B_KV_EMPTY = 12, B_S_FULL = 24, B_S_EMPTY = 26, B_P_EMPTY = 28,
+constexpr int B_KV_FULL = 0, B_KV_EMPTY = 12, B_S_FULL = 24, B_S_EMPTY = 26, B_P_EMPTY = 28,  // KV: 4 used
               B_QROPE_FULL = 30, B_Q_READY = 31, B_S_DRAIN = 32;
 // O side
 constexpr int B_V_FULL = 33, B_V_EMPTY = 37, B_P_FULL = 41, B_READY = 43, B_PV_DONE = 45,
@@ -144,6 +150,18 @@ __device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parit
   }
 }
 
+// Warp-wide bounded wait: lane 0 polls the barrier and the warp then syncs,
+// so one thread per warp (not 32) spins on the barrier while the TMA engine
+// and the tensor core share this SM's shared memory. __syncwarp orders lane
+// 0's acquire before the other lanes' reads. Call with the full warp.
+__device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(c, bar, parity, drain);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
 __global__ void __launch_bounds__(THREADS, 1) __cluster_dims__(2, 1, 1)
 verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_v,
                  const __grid_constant__ CUtensorMap tmap_q, const VerifyArgs a, const VerifyPlan p) {
@@ -178,7 +196,7 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   if (threadIdx.x == 0) {
     *c.abort_flag = 0;
     if (rank == 0) {
-      for (int i = 0; i < KV_SLOTS; ++i) {
+      for (int i = 0; i < KV_STAGES; ++i) {
         mbar_init(c.bar(B_KV_FULL + i), 1);
         mbar_init(c.bar(B_KV_EMPTY + i), 1);
       }
@@ -229,64 +247,72 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   if (rank == 0) {
     // ======================================================= S side (CTA 0)
     if (warp == 0 && lane == 0) {
-      // ---------------- producer. Ring position pos holds slot pos % 12; the
-      // q_lat blocks take positions 0-7, KV block u (tile u/9, dims 64*(u%9))
-      // takes position u + 8.
-      const int n_blocks = n_tiles * QK_BLOCKS;
+      // ---------------- producer. Stage use number pos goes to ring stage
+      // pos % 4: q_lat fills uses 0-2 (stages 0-2), KV stage g (three dim-
+      // blocks of tile g/3) is use g + 3.
+      const int n_stg = n_tiles * STAGES_PER_TILE;
       int issued = 0;
-      bool ok = true;
       if (n_tiles > 0) {
         const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
-        for (int blk = 0; blk < QLAT_BLOCKS; ++blk) {
-          mbar_arrive_expect_tx(c.bar(B_KV_FULL + blk), QBLOCK_BYTES);
-          tma_load_2d(base + OFF_RING + blk * KBLOCK_BYTES, &tmap_q, c.bar(B_KV_FULL + blk), blk * 64, qy);
+        for (int st = 0; st < Q_STAGES; ++st) {
+          const int nb = min(STAGE_BLOCKS, QLAT_BLOCKS - st * STAGE_BLOCKS);
+          mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), nb * QBLOCK_BYTES);
+          for (int e = 0; e < nb; ++e) {
+            const int blk = st * STAGE_BLOCKS + e;
+            tma_load_2d(base + OFF_RING + blk * KBLOCK_BYTES, &tmap_q, c.bar(B_KV_FULL + st), blk * 64, qy);
+          }
         }
         mbar_arrive_expect_tx(c.bar(B_QROPE_FULL), QBLOCK_BYTES);
         tma_load_2d(base + OFF_QROPE, &tmap_q, c.bar(B_QROPE_FULL), QLAT_BLOCKS * 64, qy);
       }
-      for (int u = 0; u < n_blocks; ++u) {
-        const int pos = u + KV_FIRST, slot = pos % KV_SLOTS;
-        if (!wait_bar(c, c.bar(B_KV_EMPTY + slot), ((pos / KV_SLOTS) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(c.bar(B_KV_FULL + slot), KBLOCK_BYTES);
-        const int tile = u / QK_BLOCKS, blk = u - tile * QK_BLOCKS;
-        tma_load_2d(base + OFF_RING + slot * KBLOCK_BYTES, &tmap_kv, c.bar(B_KV_FULL + slot), blk * 64,
-                    (int32_t)(kv_base + k_lo + tile * KEYS));
-        issued = u + 1;
+      for (int g = 0; g < n_stg; ++g) {
+        const int pos = g + Q_STAGES, st = pos % KV_STAGES;
+        if (!wait_bar(c, c.bar(B_KV_EMPTY + st), ((pos / KV_STAGES) & 1) ^ 1)) break;
+        mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), STAGE_BLOCKS * KBLOCK_BYTES);
+        const int tile = g / STAGES_PER_TILE, blk0 = (g % STAGES_PER_TILE) * STAGE_BLOCKS;
+        const int32_t y = (int32_t)(kv_base + k_lo + tile * KEYS);
+        for (int e = 0; e < STAGE_BLOCKS; ++e)
+          tma_load_2d(base + OFF_RING + (st * STAGE_BLOCKS + e) * KBLOCK_BYTES, &tmap_kv, c.bar(B_KV_FULL + st),
+                      (blk0 + e) * 64, y);
+        issued = g + 1;
       }
-      (void)ok;
       // retire copies still in flight (normally none: the MMA consumed them)
       if (n_tiles > 0) wait_bar(c, c.bar(B_QROPE_FULL), 0, true);
-      for (int u = max(0, issued - KV_SLOTS); u < issued; ++u) {
-        const int pos = u + KV_FIRST;
-        wait_bar(c, c.bar(B_KV_FULL + pos % KV_SLOTS), (pos / KV_SLOTS) & 1, true);
+      for (int g = max(0, issued - KV_STAGES); g < issued; ++g) {
+        const int pos = g + Q_STAGES;
+        wait_bar(c, c.bar(B_KV_FULL + pos % KV_STAGES), (pos / KV_STAGES) & 1, true);
       }
     } else if (warp == 1 && lane == 0) {
       // ---------------- QK^T MMA issuer: S[128 x 128] = Q[128 x 576] . K^T
       bool ok = n_tiles == 0 || (wait_bar(c, c.bar(B_Q_READY), 0) && wait_bar(c, c.bar(B_QROPE_FULL), 0));
       tc_fence_after();
-      // the q_lat staging blocks (ring slots 0-7) are free once Q is in TMEM
+      // the q_lat staging stages (0-2) are free once Q is in TMEM
       if (ok && n_tiles > 0)
-        for (int blk = 0; blk < QLAT_BLOCKS; ++blk) mbar_arrive(c.bar(B_KV_EMPTY + blk));
+        for (int st = 0; st < Q_STAGES; ++st) mbar_arrive(c.bar(B_KV_EMPTY + st));
       for (int i = 0; ok && i < n_tiles; ++i) {
         const int sb = i % S_BUFS;
         if (!wait_bar(c, c.bar(B_S_EMPTY + sb), ((i / S_BUFS) & 1) ^ 1)) break;
         tc_fence_after();
         const uint32_t d = tmem + TMEM_S_COL + sb * KEYS;
-        for (int blk = 0; ok && blk < QK_BLOCKS; ++blk) {
-          const int pos = i * QK_BLOCKS + blk + KV_FIRST, slot = pos % KV_SLOTS;
-          if (!wait_bar(c, c.bar(B_KV_FULL + slot), (pos / KV_SLOTS) & 1)) { ok = false; break; }
+        for (int gs = 0; ok && gs < STAGES_PER_TILE; ++gs) {
+          const int pos = i * STAGES_PER_TILE + gs + Q_STAGES, st = pos % KV_STAGES;
+          if (!wait_bar(c, c.bar(B_KV_FULL + st), (pos / KV_STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kb = base + OFF_RING + slot * KBLOCK_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = sw128_desc(kb + kk * 32, 16, 1024);
-            const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
-            if (blk < QLAT_BLOCKS)
-              mma_ts(d, tmem + TMEM_QLAT_COL + (blk * 4 + kk) * 8, bdesc, IDESC_QK, acc);
-            else
-              mma_ss(d, sw128_desc(base + OFF_QROPE + kk * 32, 16, 1024), bdesc, IDESC_QK, acc);
+          for (int e = 0; e < STAGE_BLOCKS; ++e) {
+            const int blk = gs * STAGE_BLOCKS + e;
+            const uint32_t kb = base + OFF_RING + (st * STAGE_BLOCKS + e) * KBLOCK_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bdesc = sw128_desc(kb + kk * 32, 16, 1024);
+              const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
+              if (blk < QLAT_BLOCKS)
+                mma_ts(d, tmem + TMEM_QLAT_COL + (blk * 4 + kk) * 8, bdesc, IDESC_QK, acc);
+              else
+                mma_ss(d, sw128_desc(base + OFF_QROPE + kk * 32, 16, 1024), bdesc, IDESC_QK, acc);
+            }
           }
-          tc_commit(c.bar(B_KV_EMPTY + slot));
+          tc_commit(c.bar(B_KV_EMPTY + st));
         }
         if (!ok) break;
         tc_commit(c.bar(B_S_FULL + sb));
@@ -303,8 +329,8 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
       bool ok = true;
       if (n_tiles > 0) {
-        // q_lat row (TMA-staged, 128B-swizzled, ring slots 0-7) -> TMEM columns [0, 256)
-        for (int blk = 0; blk < QLAT_BLOCKS; ++blk) ok = ok && wait_bar(c, c.bar(B_KV_FULL + blk), 0);
+        // q_lat row (TMA-staged, 128B-swizzled, first 8 ring blocks) -> TMEM columns [0, 256)
+        for (int st = 0; st < Q_STAGES; ++st) ok = wait_warp(c, c.bar(B_KV_FULL + st), 0) && ok;
         if (__all_sync(0xffffffffu, ok)) {
 #pragma unroll 1
           for (int blk = 0; blk < QLAT_BLOCKS; ++blk) {
@@ -333,7 +359,7 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       const uint32_t peer_pfull = mapa(c.bar(B_P_FULL), 1);
       for (int i = 0; i < n_tiles; ++i) {
         const int sb = i % S_BUFS;
-        ok = ok && wait_bar(c, c.bar(B_S_FULL + sb), (i / S_BUFS) & 1);
+        ok = wait_warp(c, c.bar(B_S_FULL + sb), (i / S_BUFS) & 1) && ok;
         const bool wok = __all_sync(0xffffffffu, ok);     // tcgen05.ld is warp-aligned
         uint32_t sv[KEYS];
         if (wok) {
@@ -385,7 +411,7 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
         // hand P (and the rescale factor) to the O side with async stores
         const int slot = i % NP;
-        ok = ok && wait_bar(c, c.bar(B_P_EMPTY + slot), ((i / NP) & 1) ^ 1);
+        ok = wait_warp(c, c.bar(B_P_EMPTY + slot), ((i / NP) & 1) ^ 1) && ok;
         const uint32_t pslot = peer_p + slot * P_SLOT_BYTES;
         const uint32_t pbar = peer_pfull + slot * 8;
         float lsum = 0.f;
@@ -471,8 +497,11 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         const int slot = i % NP;
         if (!wait_bar(c, c.bar(B_PV_DONE + slot), (i / NP) & 1)) break;
         if (i + NP < n_tiles) {
+          // relaxed: the MMAs that read the slot are complete (commit observed),
+          // and the slot's next bytes arrive by complete_tx; a release-ordered
+          // remote arrive costs ~4x more on this part (measured)
           mbar_arrive_expect_tx(c.bar(B_P_FULL + slot), P_MSG_BYTES);
-          mbar_arrive_remote(peer_pempty + slot * 8);
+          mbar_arrive_remote_relaxed(peer_pempty + slot * 8);
         }
       }
     } else if (warp >= WG_FIRST_WARP) {
@@ -485,12 +514,12 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       bool ok = true;
       for (int i = 0; i < n_tiles; ++i) {
         const int slot = i % NP;
-        ok = ok && wait_bar(c, c.bar(B_P_FULL + slot), (i / NP) & 1);
+        ok = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1) && ok;
         const float al = *reinterpret_cast<volatile float*>(smem + OFF_P + slot * P_SLOT_BYTES + P_BYTES + r * 4);
         const bool need = ok && i > 0 && al != 1.f;
         if (__any_sync(0xffffffffu, need)) {
           // O must be quiescent: wait for tile i-1's MMAs, then scale the rows
-          if (ok) ok = wait_bar(c, c.bar(B_PV_DONE + (i - 1) % NP), ((i - 1) / NP) & 1);
+          ok = wait_warp(c, c.bar(B_PV_DONE + (i - 1) % NP), ((i - 1) / NP) & 1) && ok;
           if (__all_sync(0xffffffffu, ok)) {
             __syncwarp();
             tc_fence_after();
@@ -514,10 +543,10 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       bool have_o = n_tiles > 0;
       if (have_o) {
         const int i = n_tiles - 1;
-        have_o = wait_bar(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
+        have_o = wait_warp(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
       }
       have_o = __all_sync(0xffffffffu, have_o);
-      ok = wait_bar(c, c.bar(B_STATS), 0) && ok && have_o == (n_tiles > 0);
+      ok = wait_warp(c, c.bar(B_STATS), 0) && ok && have_o == (n_tiles > 0);
       __syncwarp();
       tc_fence_after();
       const float l = *reinterpret_cast<volatile float*>(smem + OFF_STATS + r * 4);
@@ -611,6 +640,32 @@ cudaError_t launch_verify_tc(const VerifyArgs& a, const VerifyPlan& p, cudaStrea
   }
   verify_tc_kernel<<<2 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, a, p);
   return cudaGetLastError();
+}
+
+int tc1_max_active_clusters() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
+  if (cached[dev] > 0) return cached[dev];
+  if (cudaFuncSetAttribute(verify_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 64);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, verify_tc_kernel, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
+  cached[dev] = n;
+  return n;
 }
 
 }  // namespace kdv

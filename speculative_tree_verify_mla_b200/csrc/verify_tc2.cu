@@ -1,0 +1,699 @@
+// verify_tc2.cu -- tensor-core tree-verify MLA attention on 2-SM MMAs
+// (tcgen05.mma cta_group::2, TMEM accumulators, TMA-staged operands).
+//
+// Same operation as verify_tc.cu (page "The Architecture of Diagnosis",
+// section "Phase 1: Custom CUDA Kernels", item 2; latent dims from page "From
+// Diagnosis to Deployment", section "The Second Thread"): per query row,
+// s_j = scale (q_lat . c_kv[j] + q_rope . k_rope[j]), a softmax over the keys
+// the row's tree node may see, o_lat = sum_j p_j c_kv[j], and the split's LSE.
+//
+// Why 2-SM pairs. Staging a 128-key x 576-dim KV tile for one 128-row MMA
+// needs about as many shared-memory bytes per cycle for the TMA writes as the
+// tensor core reads back, and together they exceed what one SM's shared
+// memory delivers. In a cta_group::2 MMA the B operand is split across the
+// two SMs of a pair, so each SM stages and reads only half of it.
+//
+// One work item = 256 query rows of one request and one key split, on a
+// 4-CTA cluster:
+//   CTA 0 + CTA 1 ("S pair"): S = Q K^T with M=256 (rows 0-127 in CTA 0,
+//     128-255 in CTA 1), N=256 keys, K=576. Each CTA holds its rows' q_lat in
+//     TMEM (256 columns), its S tile in the other 256 columns, q_rope in
+//     shared memory, and stages the KV rows of its half of the keys (128 of
+//     every 256) through a 48 KB x 4 ring. CTA 0 issues the MMAs. Two softmax
+//     warpgroups per CTA (one row per thread, keys 0-127 and 128-255 of the
+//     tile) share the row maximum through shared memory, and each pushes its
+//     bf16 P half to the partner CTA on the O side with st.async.
+//   CTA 2 + CTA 3 ("O pair"): O += P V with M=256, N=256 (two MMAs per 16
+//     keys), K=16, per 128-key P tile. O (128 rows x 512 fp32) fills each
+//     CTA's TMEM; each CTA stages 256 of the 512 V dims (the half of each
+//     N=256 column range the MMA expects from it) through a 16 KB x 8 ring.
+//     CTA 2 issues the MMAs.
+//
+// Every MMA is N=256: with the TMA stream running beside it, N=128 MMAs on
+// this part leave ~35 cycles per instruction unhidden, N=256 ones do not
+// (measured). Cross-CTA arrivals are relaxed (see arrive_on).
+//
+// Softmax, lazy rescale, bounded waits and the split epilogue are as in
+// verify_tc.cu.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kdv_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace kdv {
+namespace {
+
+using namespace ptx;
+
+constexpr int DQ = 576, DC = 512;
+constexpr int ROWS = 128;                           // rows per CTA (256 per pair)
+constexpr int STILE = 2 * TC_KEYS;                  // 256 keys per S tile (QK^T N)
+constexpr int KEYS = TC_KEYS;                       // 128 keys per P tile
+constexpr int HKEYS = STILE / 2;                    // keys of an S tile staged per S CTA
+constexpr int VKEYS = 32;                           // keys per V stage
+constexpr int KBLOCK_BYTES = HKEYS * 128;           // 128 keys x 64 dims, swizzled (16 KB)
+constexpr int VBLOCK_BYTES = VKEYS * 128;           // 32 keys x 64 dims (4 KB)
+constexpr int QBLOCK_BYTES = ROWS * 128;            // 128 rows x 64 dims (16 KB)
+constexpr int QK_BLOCKS = DQ / 64;                  // 9 (8 latent + 1 rope)
+constexpr int QLAT_BLOCKS = 8;
+constexpr int V_LOCAL_BLOCKS = 4;                   // V dim-blocks per O CTA per stage
+constexpr int STAGE_BLOCKS = 3;
+constexpr int KV_STAGES = 4;
+constexpr int KV_STAGE_BYTES = STAGE_BLOCKS * KBLOCK_BYTES;   // 48 KB
+constexpr int Q_STAGES = 3;                         // ring stages covering q_lat staging
+constexpr int STAGES_PER_TILE = QK_BLOCKS / STAGE_BLOCKS;
+constexpr int V_STAGES = 8;
+constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
+constexpr int NP = 2;
+constexpr int P_BYTES = ROWS * KEYS * 2;
+constexpr int P_KBLOCK_BYTES = ROWS * 128;
+constexpr int P_MSG_BYTES = P_BYTES + ROWS * 4;
+constexpr int P_SLOT_BYTES = 33792;
+constexpr int STATS_BYTES = 2 * ROWS * 4;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_QLAT_COL = 0;
+constexpr uint32_t TMEM_S_COL = 256;
+constexpr float TAU = 8.0f;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr uint64_t TIMEOUT_NS = 1000000000ull;
+static_assert(QK_BLOCKS % STAGE_BLOCKS == 0, "stage geometry");
+static_assert(QLAT_BLOCKS * QBLOCK_BYTES <= Q_STAGES * KV_STAGE_BYTES, "q_lat staging");
+static_assert(Q_STAGES < KV_STAGES, "ring too small");
+
+// Shared-memory layout (same offsets in all four CTAs; mapa() relies on it).
+//   S CTAs: [0, 196608) KV ring (4 x 48 KB; q_lat staging in the first 128 KB
+//           at start-up); [196608, 212992) q_rope; row-max / row-sum exchange.
+//   O CTAs: [0, 131072) V ring (8 x 16 KB); P slots; final stats.
+constexpr int OFF_RING = 0;
+constexpr int OFF_QROPE = KV_STAGES * KV_STAGE_BYTES;
+constexpr int OFF_XCHG = OFF_QROPE + QBLOCK_BYTES;           // float [2][2][128] + [128] (S side)
+constexpr int XCHG_BYTES = 5 * ROWS * 4;
+constexpr int OFF_P = V_STAGES * V_STAGE_BYTES;
+constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
+constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
+static_assert(OFF_STATS + STATS_BYTES <= OFF_MISC, "O-side buffers overlap misc");
+constexpr int OFF_BAR = OFF_MISC;
+constexpr int NUM_BARS = 48;
+constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int SMEM_USED = OFF_ABORT + 12;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of shared memory");
+
+// Barrier slots (each CTA initialises the slots its role uses).
+// S pair. KV_FULL, S_EMPTY, QROPE_FULL and Q_READY are used in CTA 0 only
+// (the MMA issuer's barriers); the others in both S CTAs.
+constexpr int B_KV_FULL = 0, B_KV_EMPTY = 4, B_S_FULL = 8, B_S_EMPTY = 9, B_P_EMPTY = 10,
+              B_QLAT_FULL = 12, B_QROPE_FULL = 13, B_Q_READY = 14, B_S_DRAIN = 15;
+// O pair. V_FULL, READY and O_DRAIN in CTA 2 only.
+constexpr int B_V_FULL = 16, B_V_EMPTY = 24, B_P_FULL = 32, B_READY = 34, B_PV_DONE = 36,
+              B_STATS = 38, B_O_DRAIN = 39;
+static_assert(B_O_DRAIN < NUM_BARS, "barrier slots");
+
+constexpr uint16_t S_PAIR = 0x3, O_PAIR = 0xC;     // cluster CTA masks
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(256, 256, false, false);
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(256, 256, false, true);
+
+constexpr int THREADS = 384;
+constexpr int WG_FIRST_WARP = 4;      // warps 4-7: softmax keys 0-127 / O-side rescale + epilogue
+constexpr int WG2_FIRST_WARP = 8;     // warps 8-11: softmax keys 128-255 (S side)
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+struct Ctx {
+  uint32_t base;
+  volatile uint32_t* abort_flag;
+  int32_t* d_err;
+  __device__ uint32_t bar(int i) const { return base + OFF_BAR + 8 * i; }
+};
+
+__device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (!drain && *c.abort_flag) return false;
+      if (globaltimer() - t0 > TIMEOUT_NS) {
+        *c.abort_flag = 1;
+        record_error(c.d_err, KDV_DERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-wide bounded wait: lane 0 polls the barrier and the warp then syncs,
+// so one thread per warp (not 32) spins on the barrier while the TMA engine
+// and the tensor core share this SM's shared memory. __syncwarp orders lane
+// 0's acquire before the other lanes' reads. Call with the full warp.
+__device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(c, bar, parity, drain);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// Arrive on barrier `bar` (local offset) of CTA `rank`: a local arrive when
+// it is this CTA, else a relaxed remote arrive. No cross-CTA arrival here
+// publishes generic-proxy data: each follows tcgen05.ld / tcgen05.st work the
+// thread has already waited for (tcgen05.wait) or guards bytes that reach the
+// other side through complete_tx. A release-ordered remote arrive costs
+// ~1800 cycles on this part against ~440 for a relaxed one (measured), enough
+// to starve the pipeline.
+__device__ __forceinline__ void arrive_on(uint32_t bar, uint32_t rank, uint32_t my_rank) {
+  if (rank == my_rank) mbar_arrive(bar);
+  else mbar_arrive_remote_relaxed(mapa(bar, rank));
+}
+
+__global__ void __launch_bounds__(THREADS, 1) __cluster_dims__(4, 1, 1)
+verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_v,
+                  const __grid_constant__ CUtensorMap tmap_q, const VerifyArgs a, const VerifyPlan p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t rank = cluster_ctarank();
+  const bool s_side = rank < 2;
+  const uint32_t half = rank & 1;                 // which 128 rows (and which operand half)
+  const bool leader = half == 0;                  // CTA 0 / CTA 2 issue the pair's MMAs
+  const uint32_t lead_rank = rank & ~1u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  Ctx c;
+  c.base = base;
+  c.abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_ABORT);
+  c.d_err = a.d_err;
+
+  // ---- work item ---------------------------------------------------------
+  const int item = blockIdx.x >> 2;
+  const int b = plan_request(p, item);
+  const int local = item - p.item_base[b];
+  const int split = local / p.tiles[b];
+  const int rt = local - split * p.tiles[b];
+  const int H = p.H, L = p.L[b], Tn = p.T[b];
+  const int n_keys = L + Tn;
+  const int rows_b = Tn * H;
+  const int row0 = rt * (2 * ROWS) + (int)half * ROWS;   // this CTA's first row
+  const int k_lo = min(split * p.chunk[b], n_keys);
+  const int k_hi = min(k_lo + p.chunk[b], n_keys);
+  const int n_stiles = (k_hi - k_lo + STILE - 1) / STILE;
+  const int n_ptiles = 2 * n_stiles;
+  const int64_t kv_base = a.kv_off[b];
+
+  // ---- setup -------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    *c.abort_flag = 0;
+    if (s_side) {
+      for (int i = 0; i < KV_STAGES; ++i) {
+        mbar_init(c.bar(B_KV_FULL + i), 1);
+        mbar_init(c.bar(B_KV_EMPTY + i), 1);
+      }
+      mbar_init(c.bar(B_S_FULL), 1);
+      mbar_init(c.bar(B_S_EMPTY), 4 * ROWS);             // both warpgroups of both S CTAs
+      for (int i = 0; i < NP; ++i) mbar_init(c.bar(B_P_EMPTY + i), 1);
+      mbar_init(c.bar(B_QLAT_FULL), 1);
+      mbar_init(c.bar(B_QROPE_FULL), 1);
+      mbar_init(c.bar(B_Q_READY), 2 * ROWS);
+      mbar_init(c.bar(B_S_DRAIN), 1);
+      // KV_FULL phase k of ring stage st belongs to ring use st + 4k; the
+      // stages that hold q_lat at start-up (uses 0-2) carry no KV, so their
+      // first phase is completed here
+      for (int st = 0; st < Q_STAGES; ++st) mbar_arrive(c.bar(B_KV_FULL + st));
+      if (leader) {
+        if (a.prefix_len != nullptr && a.prefix_len[b] != L) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+        if (a.tree_off != nullptr && a.tree_off[b] != p.tree_base[b]) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+        if ((int64_t)a.kv_off[b + 1] - kv_base < (int64_t)n_keys) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+      }
+      tma_prefetch_desc(&tmap_kv);
+      tma_prefetch_desc(&tmap_q);
+    } else {
+      for (int i = 0; i < V_STAGES; ++i) {
+        mbar_init(c.bar(B_V_FULL + i), 1);
+        mbar_init(c.bar(B_V_EMPTY + i), 1);
+      }
+      for (int i = 0; i < NP; ++i) {
+        mbar_init(c.bar(B_P_FULL + i), 1);
+        mbar_init(c.bar(B_READY + i), 2 * ROWS);
+        mbar_init(c.bar(B_PV_DONE + i), 1);
+      }
+      mbar_init(c.bar(B_STATS), 1);
+      mbar_init(c.bar(B_O_DRAIN), 1);
+      for (int i = 0; i < NP; ++i) mbar_arrive_expect_tx(c.bar(B_P_FULL + i), P_MSG_BYTES);
+      mbar_arrive_expect_tx(c.bar(B_STATS), STATS_BYTES);
+      tma_prefetch_desc(&tmap_v);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc2(base + OFF_TMEM, TMEM_COLS);
+    tmem_relinquish2();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+
+  if (s_side) {
+    // ======================================================= S pair
+    if (warp == 0 && lane == 0) {
+      // ---------------- producer (both S CTAs): q_lat staging (local), q_rope
+      // and this CTA's 128 of every 256 KV rows (counted on the leader's barriers)
+      const int n_stg = n_stiles * STAGES_PER_TILE;
+      int issued = 0;
+      if (n_stiles > 0) {
+        const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
+        mbar_arrive_expect_tx(c.bar(B_QLAT_FULL), QLAT_BLOCKS * QBLOCK_BYTES);
+        for (int blk = 0; blk < QLAT_BLOCKS; ++blk)
+          tma_load_2d(base + OFF_RING + blk * QBLOCK_BYTES, &tmap_q, c.bar(B_QLAT_FULL), blk * 64, qy);
+        if (leader) mbar_arrive_expect_tx(c.bar(B_QROPE_FULL), 2 * QBLOCK_BYTES);
+        tma_load_2d_pair(base + OFF_QROPE, &tmap_q, mapa(c.bar(B_QROPE_FULL), lead_rank), QLAT_BLOCKS * 64, qy);
+      }
+      for (int g = 0; g < n_stg; ++g) {
+        const int pos = g + Q_STAGES, st = pos % KV_STAGES;
+        if (!wait_bar(c, c.bar(B_KV_EMPTY + st), ((pos / KV_STAGES) & 1) ^ 1)) break;
+        if (leader) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KV_STAGE_BYTES);
+        const int tile = g / STAGES_PER_TILE, blk0 = (g % STAGES_PER_TILE) * STAGE_BLOCKS;
+        const int32_t y = (int32_t)(kv_base + k_lo + tile * STILE + (int)half * HKEYS);
+        const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
+        for (int e = 0; e < STAGE_BLOCKS; ++e)
+          tma_load_2d_pair(base + OFF_RING + st * KV_STAGE_BYTES + e * KBLOCK_BYTES, &tmap_kv, fb, (blk0 + e) * 64, y);
+        issued = g + 1;
+      }
+      if (n_stiles > 0) wait_bar(c, c.bar(B_QLAT_FULL), 0, true);
+      if (leader) {
+        // retire copies in flight (both halves count on the leader's barriers)
+        if (n_stiles > 0) wait_bar(c, c.bar(B_QROPE_FULL), 0, true);
+        for (int g = max(0, issued - KV_STAGES); g < issued; ++g) {
+          const int pos = g + Q_STAGES;
+          wait_bar(c, c.bar(B_KV_FULL + pos % KV_STAGES), (pos / KV_STAGES) & 1, true);
+        }
+      }
+    } else if (warp == 1 && lane == 0 && leader) {
+      // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T
+      bool ok = n_stiles == 0 || (wait_bar(c, c.bar(B_Q_READY), 0) && wait_bar(c, c.bar(B_QROPE_FULL), 0));
+      tc_fence_after();
+      if (ok && n_stiles > 0) {
+        // the q_lat staging stages are free in both S CTAs once Q is in TMEM
+        for (int st = 0; st < Q_STAGES; ++st) {
+          mbar_arrive(c.bar(B_KV_EMPTY + st));
+          mbar_arrive_remote_relaxed(mapa(c.bar(B_KV_EMPTY + st), lead_rank + 1));
+        }
+      }
+      const uint32_t d = tmem + TMEM_S_COL;
+      for (int i = 0; ok && i < n_stiles; ++i) {
+        if (!wait_bar(c, c.bar(B_S_EMPTY), (i & 1) ^ 1)) break;
+        tc_fence_after();
+        for (int gs = 0; ok && gs < STAGES_PER_TILE; ++gs) {
+          const int pos = i * STAGES_PER_TILE + gs + Q_STAGES, st = pos % KV_STAGES;
+          if (!wait_bar(c, c.bar(B_KV_FULL + st), (pos / KV_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int e = 0; e < STAGE_BLOCKS; ++e) {
+            const int blk = gs * STAGE_BLOCKS + e;
+            const uint32_t kb = base + OFF_RING + st * KV_STAGE_BYTES + e * KBLOCK_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bdesc = sw128_desc(kb + kk * 32, 16, 1024);
+              const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
+              if (blk < QLAT_BLOCKS)
+                mma2_ts(d, tmem + TMEM_QLAT_COL + (blk * 4 + kk) * 8, bdesc, IDESC_QK, acc);
+              else
+                mma2_ss(d, sw128_desc(base + OFF_QROPE + kk * 32, 16, 1024), bdesc, IDESC_QK, acc);
+            }
+          }
+          tc_commit2_mc(c.bar(B_KV_EMPTY + st), S_PAIR);
+        }
+        if (!ok) break;
+        tc_commit2_mc(c.bar(B_S_FULL), S_PAIR);
+      }
+      tc_commit2_mc(c.bar(B_S_DRAIN), (uint16_t)(1u << rank));
+      wait_bar(c, c.bar(B_S_DRAIN), 0, true);
+    } else if (warp >= WG_FIRST_WARP) {
+      // ---------------- softmax warpgroups (both S CTAs): thread <-> row;
+      // warpgroup hw takes keys [128*hw, 128*hw + 128) of every S tile
+      const int hw = warp >= WG2_FIRST_WARP ? 1 : 0;
+      const int sp = warp & 3;
+      const int r = sp * 32 + lane;
+      const int row = row0 + r;
+      const bool valid = row < rows_b;
+      const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+      float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);   // [2 parity][2 hw][128] (+ final sums)
+      bool ok = true;
+      if (n_stiles > 0 && hw == 0) {
+        // q_lat row (TMA-staged, 128B-swizzled) -> TMEM columns [0, 256)
+        ok = wait_warp(c, c.bar(B_QLAT_FULL), 0);
+        if (__all_sync(0xffffffffu, ok)) {
+#pragma unroll 1
+          for (int blk = 0; blk < QLAT_BLOCKS; ++blk) {
+            uint32_t v[32];
+            const uint8_t* rowp = smem + OFF_RING + blk * QBLOCK_BYTES + r * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint4 u4 = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (r & 7)) << 4));
+              v[4 * ch + 0] = u4.x;
+              v[4 * ch + 1] = u4.y;
+              v[4 * ch + 2] = u4.z;
+              v[4 * ch + 3] = u4.w;
+            }
+            __syncwarp();
+            tmem_st32(tmem + lane_base + TMEM_QLAT_COL + blk * 32, v);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        arrive_on(c.bar(B_Q_READY), lead_rank, rank);
+      }
+      const uint64_t mask_t = valid ? a.mask[p.tree_base[b] + row / H] : 0ull;
+      const float sl2 = a.scale * LOG2E;
+      float m_run = -INFINITY, l_part = 0.f;
+      const uint32_t o_rank = 2 + half;                       // this CTA's O partner
+      const uint32_t pslot = mapa(base + OFF_P, o_rank) + hw * P_SLOT_BYTES;
+      const uint32_t pbar = mapa(c.bar(B_P_FULL), o_rank) + hw * 8;
+      for (int i = 0; i < n_stiles; ++i) {
+        ok = wait_warp(c, c.bar(B_S_FULL), i & 1) && ok;
+        const bool wok = __all_sync(0xffffffffu, ok);
+        uint32_t sv[KEYS];
+        if (wok) {
+          __syncwarp();
+          tc_fence_after();
+          const uint32_t sa = tmem + lane_base + TMEM_S_COL + hw * KEYS;
+          tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(sv));
+          tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+          tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+          tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+          tmem_wait_ld();
+          tc_fence_before();
+          arrive_on(c.bar(B_S_EMPTY), lead_rank, rank);
+        } else {
+#pragma unroll
+          for (int k = 0; k < KEYS; ++k) sv[k] = 0u;
+        }
+        ok = ok && wok;
+        const int key0 = k_lo + i * STILE + hw * KEYS;
+        float m_half = -INFINITY;
+        if (valid && key0 + KEYS <= min(L, k_hi)) {
+#pragma unroll
+          for (int k = 0; k < KEYS; ++k) {
+            const float xk = __uint_as_float(sv[k]) * sl2;
+            sv[k] = __float_as_uint(xk);
+            m_half = fmaxf(m_half, xk);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < KEYS; ++k) {
+            const int j = key0 + k;
+            bool vis = valid && j < k_hi;
+            if (j >= L) vis = vis && ((mask_t >> ((j - L) & 63)) & 1ull);
+            const float xk = vis ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
+            sv[k] = __float_as_uint(xk);
+            m_half = fmaxf(m_half, xk);
+          }
+        }
+        // row max of the whole 256-key tile from both warpgroups
+        volatile float* xm = xchg + (i & 1) * 2 * ROWS;
+        xm[hw * ROWS + r] = m_half;
+        named_bar_sync(1, 2 * 128);
+        const float m_tile = fmaxf(m_half, xm[(hw ^ 1) * ROWS + r]);
+        float alpha = 1.f;
+        if (m_tile > m_run + TAU || (m_run == -INFINITY && m_tile != -INFINITY)) {
+          if (m_run != -INFINITY) {
+            alpha = ex2(m_run - m_tile);
+            l_part *= alpha;
+          }
+          m_run = m_tile;
+        }
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        // P tile 2i + hw goes to O-side slot hw
+        ok = wait_warp(c, c.bar(B_P_EMPTY + hw), (i & 1) ^ 1) && ok;
+        float lsum = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < KEYS / 8; ++ch) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float p0 = ex2(__uint_as_float(sv[8 * ch + 2 * q]) - m_use);
+            const float p1 = ex2(__uint_as_float(sv[8 * ch + 2 * q + 1]) - m_use);
+            lsum += p0 + p1;
+            w[q] = pack_bf16x2(p0, p1);
+          }
+          const int kb = ch >> 3, piece = ch & 7;
+          if (ok)
+            st_async_v4(pslot + kb * P_KBLOCK_BYTES + r * 128 + ((piece ^ (r & 7)) << 4), w[0], w[1], w[2],
+                        w[3], pbar);
+        }
+        l_part += lsum;
+        // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
+        if (ok) st_async_f32(pslot + P_BYTES + r * 4, hw == 0 ? alpha : 1.f, pbar);
+      }
+      // final row statistics (sum of both halves) for the O side's epilogue
+      volatile float* xs = xchg + 4 * ROWS;
+      named_bar_sync(1, 2 * 128);
+      if (hw == 1) xs[r] = l_part;
+      named_bar_sync(1, 2 * 128);
+      if (hw == 0) {
+        const float l = l_part + xs[r];
+        const uint32_t peer_stats = mapa(base + OFF_STATS, o_rank);
+        const uint32_t peer_sbar = mapa(c.bar(B_STATS), o_rank);
+        st_async_f32(peer_stats + r * 4, l, peer_sbar);
+        st_async_f32(peer_stats + ROWS * 4 + r * 4, m_run, peer_sbar);
+      }
+    }
+  } else {
+    // ======================================================= O pair
+    if (warp == 0 && lane == 0) {
+      // ---------------- V producer (both O CTAs): this CTA's 256 dims of
+      // every 32 keys; local block lb holds dims 64*((lb/2)*4 + half*2 + lb%2)
+      int issued = 0;
+      const int n_sub = (KEYS / VKEYS) * n_ptiles;
+      for (int u = 0; u < n_sub; ++u) {
+        const int st = u % V_STAGES;
+        if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1)) break;
+        if (leader) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
+        const int32_t y = (int32_t)(kv_base + k_lo + u * VKEYS);
+        const uint32_t dst = base + OFF_RING + st * V_STAGE_BYTES;
+        const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
+        for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
+          const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
+          tma_load_2d_pair(dst + lb * VBLOCK_BYTES, &tmap_v, fb, gb * 64, y);
+        }
+        issued = u + 1;
+      }
+      if (leader)
+        for (int u = max(0, issued - V_STAGES); u < issued; ++u)
+          wait_bar(c, c.bar(B_V_FULL + u % V_STAGES), (u / V_STAGES) & 1, true);
+    } else if (warp == 1 && lane == 0 && leader) {
+      // ---------------- pair MMA issuer: O[256 x 512] += P[256 x 128] . V[128 x 512]
+      for (int i = 0; i < n_ptiles; ++i) {
+        const int slot = i % NP;
+        if (!wait_bar(c, c.bar(B_READY + slot), (i / NP) & 1)) break;
+        bool ok = true;
+        const uint32_t pbuf = base + OFF_P + slot * P_SLOT_BYTES;
+        for (int h = 0; ok && h < KEYS / VKEYS; ++h) {
+          const int u = (KEYS / VKEYS) * i + h, st = u % V_STAGES;
+          if (!wait_bar(c, c.bar(B_V_FULL + st), (u / V_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t vst = base + OFF_RING + st * V_STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < VKEYS / 16; ++kk) {
+            const int k = (VKEYS / 16) * h + kk;
+            const uint64_t adesc = sw128_desc(pbuf + (k >> 2) * P_KBLOCK_BYTES + (k & 3) * 32, 16, 1024);
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+              // this CTA's 128 of the 256 columns: two 64-dim blocks, LBO apart
+              const uint64_t bdesc = sw128_desc(vst + nh * 2 * VBLOCK_BYTES + kk * 2048, VBLOCK_BYTES, 1024);
+              mma2_ss(tmem + nh * 256, adesc, bdesc, IDESC_PV, (i > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit2_mc(c.bar(B_V_EMPTY + st), O_PAIR);
+        }
+        if (!ok) break;
+        tc_commit2_mc(c.bar(B_PV_DONE + slot), O_PAIR);
+      }
+      tc_commit2_mc(c.bar(B_O_DRAIN), (uint16_t)(1u << rank));
+      wait_bar(c, c.bar(B_O_DRAIN), 0, true);
+    } else if (warp == 3 && lane == 0) {
+      // ---------------- P-slot releaser (both O CTAs)
+      const uint32_t peer_pempty = mapa(c.bar(B_P_EMPTY), half);
+      for (int i = 0; i < n_ptiles; ++i) {
+        const int slot = i % NP;
+        if (!wait_bar(c, c.bar(B_PV_DONE + slot), (i / NP) & 1)) break;
+        if (i + NP < n_ptiles) {
+          mbar_arrive_expect_tx(c.bar(B_P_FULL + slot), P_MSG_BYTES);
+          mbar_arrive_remote_relaxed(peer_pempty + slot * 8);
+        }
+      }
+    } else if (warp >= WG_FIRST_WARP && warp < WG2_FIRST_WARP) {
+      // ---------------- rescale + epilogue (both O CTAs): thread <-> row
+      const int sp = warp & 3;
+      const int r = sp * 32 + lane;
+      const int row = row0 + r;
+      const bool valid = row < rows_b;
+      const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+      bool ok = true;
+      for (int i = 0; i < n_ptiles; ++i) {
+        const int slot = i % NP;
+        ok = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1) && ok;
+        fence_proxy_async_smem();      // P arrived by st.async; the pair's MMA reads it
+        const float al = *reinterpret_cast<volatile float*>(smem + OFF_P + slot * P_SLOT_BYTES + P_BYTES + r * 4);
+        const bool need = ok && i > 0 && al != 1.f;
+        if (__any_sync(0xffffffffu, need)) {
+          // O must be quiescent: wait for tile i-1's MMAs, then scale the rows
+          ok = wait_warp(c, c.bar(B_PV_DONE + (i - 1) % NP), ((i - 1) / NP) & 1) && ok;
+          if (__all_sync(0xffffffffu, ok)) {
+            __syncwarp();
+            tc_fence_after();
+            const float f = need ? al : 1.f;
+#pragma unroll 1
+            for (int cb = 0; cb < DC / 32; ++cb) {
+              uint32_t v[32];
+              tmem_ld32(tmem + lane_base + cb * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
+              tmem_st32(tmem + lane_base + cb * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+        }
+        if (ok) arrive_on(c.bar(B_READY + slot), lead_rank, rank);
+      }
+      // ---------------- epilogue: o = O / l, lse = ln2 * (m + log2 l)
+      bool have_o = n_ptiles > 0;
+      if (have_o) {
+        const int i = n_ptiles - 1;
+        have_o = wait_warp(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
+      }
+      have_o = __all_sync(0xffffffffu, have_o);
+      ok = wait_warp(c, c.bar(B_STATS), 0) && ok && have_o == (n_ptiles > 0);
+      __syncwarp();
+      tc_fence_after();
+      const float l = *reinterpret_cast<volatile float*>(smem + OFF_STATS + r * 4);
+      const float m = *reinterpret_cast<volatile float*>(smem + OFF_STATS + ROWS * 4 + r * 4);
+      const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
+      const float lse = (l > 0.f && ok) ? (m + __log2f(l)) * LN2 : -INFINITY;
+      const int64_t orow = out_row_index(p, b, split, row);
+      float* orow_ptr = a.o + orow * DC;
+#pragma unroll 1
+      for (int cb = 0; cb < DC / 32; ++cb) {
+        uint32_t v[32];
+        if (have_o) {
+          tmem_ld32(tmem + lane_base + cb * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = 0u;
+        }
+        if (valid) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float4 f;
+            f.x = __uint_as_float(v[4 * k + 0]) * inv;
+            f.y = __uint_as_float(v[4 * k + 1]) * inv;
+            f.z = __uint_as_float(v[4 * k + 2]) * inv;
+            f.w = __uint_as_float(v[4 * k + 3]) * inv;
+            *reinterpret_cast<float4*>(orow_ptr + cb * 32 + 4 * k) = f;
+          }
+        }
+      }
+      if (valid && a.lse != nullptr) a.lse[orow] = lse;
+    }
+  }
+
+  // ---- teardown ----------------------------------------------------------
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc2(tmem, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  if (a.num_slots < 1 || a.num_slots > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
+  if (p.total_rows < 1) return cudaErrorInvalidValue;
+  auto make = [&](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t pitch_elems, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)DQ, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)pitch_elems * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  CUtensorMap tmap_kv, tmap_v, tmap_q;
+  if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, HKEYS) != CUDA_SUCCESS ||
+      make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, VKEYS) != CUDA_SUCCESS ||
+      make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(verify_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  verify_tc2_kernel<<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, a, p);
+  return cudaGetLastError();
+}
+
+int tc2_max_active_clusters() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
+  if (cached[dev] > 0) return cached[dev];
+  if (cudaFuncSetAttribute(verify_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4 * 64);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, verify_tc2_kernel, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
+  cached[dev] = n;
+  return n;
+}
+
+}  // namespace kdv

@@ -1,5 +1,7 @@
-"""GPU parity of the tensor-core (tcgen05/TMEM/TMA) verify kernel vs the oracle,
-through the C ABI. Kimi/DeepSeekV3 latent dims (512 + 64), bf16 inputs."""
+"""GPU parity of the tensor-core (tcgen05/TMEM/TMA) verify kernels vs the oracle,
+through the C ABI. Kimi/DeepSeekV3 latent dims (512 + 64), bf16 inputs. Both
+kernels run every case: the 2-SM-MMA kernel (4-CTA clusters, the default) and
+the 1-SM-MMA kernel (2-CTA clusters)."""
 import math
 
 import numpy as np
@@ -10,11 +12,15 @@ from speculative_tree_verify_mla_b200 import datagen, kdv
 from tests.parity import assert_parity
 
 pytestmark = pytest.mark.gpu
-TC = kdv.KDV_IMPL_TC
 
 
-def _run(case, splits=1, partials=False):
-    dc = kdv.DeviceCase(case, impl=TC, num_splits=splits, return_partials=partials).run()
+@pytest.fixture(params=[kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_1SM], ids=["tc2sm", "tc1sm"])
+def impl(request):
+    return request.param
+
+
+def _run(case, impl, splits=1, partials=False):
+    dc = kdv.DeviceCase(case, impl=impl, num_splits=splits, return_partials=partials).run()
     out = dc.results()
     assert dc.error_flag() == 0
     return out
@@ -22,27 +28,27 @@ def _run(case, splits=1, partials=False):
 
 @pytest.mark.parametrize("L,T,H", [(700, 13, 64), (0, 5, 64), (1, 1, 64), (63, 2, 64),
                                    (64, 3, 8), (65, 16, 8), (130, 64, 4), (257, 7, 3)])
-def test_tc_single_split(L, T, H):
+def test_tc_single_split(L, T, H, impl):
     parents = [datagen.random_tree(T, np.random.default_rng(L + T))]
     case = datagen.make_case("tc", **dict(datagen.KIMI, H=H), prefix_len=[L], parents=parents,
                              seed=L * 7 + T)
-    o, lse = _run(case, splits=1)
+    o, lse = _run(case, impl, splits=1)
     o_ref, lse_ref = oracle.verify_case(case)
     assert_parity(o, lse, o_ref, lse_ref)
 
 
 @pytest.mark.parametrize("splits", [0, 3, 7])
-def test_tc_splits_merged(splits):
+def test_tc_splits_merged(splits, impl):
     case = datagen.kimi_layer_case(L=1500, T=13, seed=11)
-    o, lse = _run(case, splits=splits)
+    o, lse = _run(case, impl, splits=splits)
     o_ref, lse_ref = oracle.verify_case(case)
     assert_parity(o, lse, o_ref, lse_ref)
 
 
-def test_tc_partials_match_oracle_ranges():
+def test_tc_partials_match_oracle_ranges(impl):
     case = datagen.kimi_layer_case(L=300, T=9, seed=12)
     S = 4
-    o_part, lse_part = _run(case, splits=S, partials=True)
+    o_part, lse_part = _run(case, impl, splits=S, partials=True)
     n = 300 + 9
     c = 128 * math.ceil(n / (128 * S))
     for s in range(S):
@@ -56,30 +62,30 @@ def test_tc_partials_match_oracle_ranges():
         assert_parity(o_part[s], lse_part[s], ro, rl)
 
 
-def test_tc_batched_contiguous():
+def test_tc_batched_contiguous(impl):
     parents = [datagen.random_tree(T, np.random.default_rng(T)) for T in (9, 16, 12)]
     case = datagen.make_case("b3", **datagen.KIMI, prefix_len=[1030, 77, 400], parents=parents,
                              seed=21)
-    o, lse = _run(case, splits=0)
+    o, lse = _run(case, impl, splits=0)
     o_ref, lse_ref = oracle.verify_case(case)
     assert_parity(o, lse, o_ref, lse_ref)
 
 
-def test_tc_lazy_rescale_growing_logits():
+def test_tc_lazy_rescale_growing_logits(impl):
     """Logits that grow along the keys force the running max up by far more
     than the lazy-rescale threshold several times within one split."""
     case = datagen.kimi_layer_case(L=900, T=6, seed=13)
     ramp = np.linspace(0.2, 3.0, case.kv.shape[0], dtype=np.float32)[:, None]
     case.kv = datagen.bf16_round(case.kv * ramp)
     case = datagen.scaled_case(case, 3.0)
-    o, lse = _run(case, splits=1)
+    o, lse = _run(case, impl, splits=1)
     o_ref, lse_ref = oracle.verify_case(case)
     # inputs here are not unit-scale (|o_lat| ~ 2): only the relative bars apply
     assert_parity(o, lse, o_ref, lse_ref, max_tol=np.inf, mean_tol=np.inf)
 
 
-def test_tc_matches_simt_on_same_inputs():
+def test_tc_matches_simt_on_same_inputs(impl):
     case = datagen.kimi_layer_case(L=513, T=13, seed=14)
-    o1, l1 = _run(case, splits=2)
+    o1, l1 = _run(case, impl, splits=2)
     o2, l2 = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_SIMT, num_splits=2).run().results()
     assert_parity(o1, l1, o2, l2)
