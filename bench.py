@@ -74,21 +74,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"], source="fallback")
 
 
-def kernel_source_hash():
+TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 3: ("verify_tc_kernel", "verify_tc.cu")}
+
+
+def kernel_source_hash(src="verify_tc2.cu"):
     h = hashlib.sha256()
-    for fn in ("verify_tc.cu", "sm100_ptx.cuh", "kdv_internal.cuh"):
+    for fn in (src, "sm100_ptx.cuh", "kdv_internal.cuh"):
         with open(os.path.join(ROOT, "speculative_tree_verify_mla_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def load_traffic():
+def load_traffic(kernel, src):
     """Per-launch DRAM bytes of the TC kernel from the committed ncu summary,
-    or None when it was taken on a different kernel source."""
+    or None when it was taken on a different kernel or kernel source."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        if t.get("kernel_source_hash") == kernel_source_hash():
+        if t.get("kernel") == kernel and t.get("kernel_source_hash") == kernel_source_hash(src):
             return float(t["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -242,7 +245,7 @@ def run_gpu(args):
         kv = torch.from_numpy(c.kv).to(torch.bfloat16).to(dev)
         o = torch.empty(c.rows, 512, dtype=torch.float32, device=dev)
         lse = torch.empty(c.rows, dtype=torch.float32, device=dev)
-        p = kdv.make_params(**common, impl=kdv.KDV_IMPL_AUTO, q=q, kv=kv, num_slots=kv.shape[0],
+        p = kdv.make_params(**common, impl=args.impl_code, q=q, kv=kv, num_slots=kv.shape[0],
                             num_splits=0, return_partials=0, o=o, lse=lse, o_part=None,
                             lse_part=None, workspace=None, workspace_bytes=0)
         nbytes = kdv.kdv_verify_attn_workspace(p)
@@ -254,7 +257,7 @@ def run_gpu(args):
     o_part = torch.empty(S, c0.rows, 512, dtype=torch.float32, device=dev)
     lse_part = torch.empty(S, c0.rows, dtype=torch.float32, device=dev)
     for l, c in enumerate(cases):
-        tc_params.append(kdv.make_params(**common, impl=kdv.KDV_IMPL_TC, q=qs[l], kv=kvs[l],
+        tc_params.append(kdv.make_params(**common, impl=args.impl_code, q=qs[l], kv=kvs[l],
                                          num_slots=kvs[l].shape[0], num_splits=S, return_partials=1,
                                          o=None, lse=None, o_part=o_part, lse_part=lse_part,
                                          workspace=None, workspace_bytes=0))
@@ -375,7 +378,8 @@ def run_gpu(args):
     peaks = load_peaks()
     us_per_layer = ms_per_step * 1e3 / (NL * world)
     tc_tflops = flops / (tc_us * 1e-6) / 1e12
-    traffic = load_traffic()
+    kname, ksrc = TC_KERNEL.get(args.impl_code, TC_KERNEL[2])
+    traffic = load_traffic(kname, ksrc)
     roof_us = max(flops / (peaks["bf16_tflops"] * 1e12), kv_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
     result = {
         "metric": METRIC, "value": us_per_layer, "unit": UNIT, "n_gpus": world,
@@ -392,7 +396,7 @@ def run_gpu(args):
         "roofline_us_per_layer": roof_us,
         "frac_of_roofline": roof_us / us_per_layer,
         "eager_us_per_layer": eager_us,
-        "roofline": {"bound": "tensor", "kernel": "verify_tc_kernel", "achieved": tc_tflops,
+        "roofline": {"bound": "tensor", "kernel": kname, "achieved": tc_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tc_tflops / peaks["bf16_tflops"], "traffic": traffic,
                      "us_per_launch": tc_us, "flops_per_launch": flops,
@@ -436,7 +440,10 @@ def main():
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT)
     ap.add_argument("--impl", choices=["kdv", "reference"], default="kdv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["tc2", "tc1"], default="tc2",
+                    help="tensor-core kernel: 2-SM MMAs (default) or 1-SM MMAs")
     args = ap.parse_args()
+    args.impl_code = 2 if args.kernel == "tc2" else 3
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)
