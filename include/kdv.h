@@ -175,6 +175,30 @@ KDV_API kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* spl
 KDV_API kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream);
 
 /*
+ * kdv_verify_attn_noalloc -- kdv_verify_attn for callers that cannot allocate.
+ * The pages describe nothing like it; it is a convenience of this library.
+ * Some callers cannot give the library scratch memory: a serving engine that
+ * reserved all free device memory for its KV-cache pool at start-up, a
+ * plug-in whose host framework owns every device allocation, or a loop where
+ * an allocation on the call path costs too much. This entry point computes
+ * exactly what kdv_verify_attn computes, but keeps the split partials in a
+ * scratch array compiled into the library (KDV_NOALLOC_SCRATCH_BYTES per
+ * GPU, held by every GPU that loads the library until the process exits)
+ * and ignores p->workspace / p->workspace_bytes. It allocates no memory.
+ *   - Returns KDV_ERR_WORKSPACE when the split plan needs more scratch than
+ *     KDV_NOALLOC_SCRATCH_BYTES (kdv_verify_attn_workspace tells the size;
+ *     fewer splits or fewer requests per call fit).
+ *   - The first call on a device looks up the array's device address with
+ *     the device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents (every byte a call reads, the same call writes first). Calls
+ *     whose work overlaps on the GPU race on it: issue them on one stream or
+ *     order them.
+ */
+#define KDV_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+KDV_API kdv_status kdv_verify_attn_noalloc(const kdv_verify_params* p, void* stream);
+
+/*
  * kdv_combine -- log-sum-exp merge of S split partials (the prefix / tree-tail
  * merge of page "The Three Acts of Engineering", reference [1]):
  *   LSE = ln sum_k exp(lse_k),  o = sum_k exp(lse_k - LSE) o_k.

@@ -42,7 +42,8 @@ KDV_MAX_BATCH = 128
 # Every entry point include/kdv.h declares (checked by the CPU tests).
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
-            "kdv_combine")
+            "kdv_verify_attn_noalloc", "kdv_combine")
+KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class KdvError(RuntimeError):
@@ -97,6 +98,8 @@ def load() -> ctypes.CDLL:
         lib.kdv_verify_attn_plan.restype = c.c_int
         lib.kdv_verify_attn.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
         lib.kdv_verify_attn.restype = c.c_int
+        lib.kdv_verify_attn_noalloc.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
+        lib.kdv_verify_attn_noalloc.restype = c.c_int
         lib.kdv_combine.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int64, c.c_int32,
                                     c.c_void_p, c.c_void_p, c.c_void_p]
         lib.kdv_combine.restype = c.c_int
@@ -179,6 +182,12 @@ def kdv_verify_attn_plan(params: VerifyParams):
 
 def kdv_verify_attn(params: VerifyParams, stream=None) -> None:
     _check(load().kdv_verify_attn(ctypes.byref(params), _stream(stream)), "kdv_verify_attn")
+
+
+def kdv_verify_attn_noalloc(params: VerifyParams, stream=None) -> None:
+    """kdv_verify_attn with the library's built-in scratch instead of params.workspace."""
+    _check(load().kdv_verify_attn_noalloc(ctypes.byref(params), _stream(stream)),
+           "kdv_verify_attn_noalloc")
 
 
 def kdv_combine(o_part: torch.Tensor, lse_part: torch.Tensor, S: int, rows: int, d: int,
