@@ -68,6 +68,13 @@ def _load():
             lib.oracle_combine.argtypes = [c.c_int32, c.c_int64, c.c_int32, _f64p, _f64p,
                                            _f64p, _f64p]
             lib.oracle_combine.restype = None
+            lib.oracle_argmax.argtypes = [c.c_int64, c.c_int64, _f32p, c.c_int64, _i32p]
+            lib.oracle_argmax.restype = None
+            lib.oracle_tree_accept.argtypes = [c.c_int32, _i32p, _i32p, _i32p, _i32p,
+                                               c.POINTER(c.c_int32), c.POINTER(c.c_int32)]
+            lib.oracle_tree_accept.restype = c.c_int
+            lib.oracle_accept_commit.argtypes = [c.c_int32, c.c_int32, c.c_int32, _i32p, _i32p]
+            lib.oracle_accept_commit.restype = None
             _lib = lib
     return _lib
 
@@ -201,3 +208,71 @@ def combine(o_part, lse_part):
     lse = np.zeros(rows, dtype=np.float64)
     _load().oracle_combine(S, rows, d, o_part, lse_part, o, lse)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Greedy tree acceptance (kdv_oracle.cpp: "Greedy tree acceptance"; page "The
+# Architecture of Diagnosis", section "Phase 1: Custom CUDA Kernels", item 3).
+
+def argmax(logits) -> np.ndarray:
+    """Per-row argmax (lowest index among equal maxima, NaN never wins, all-NaN -> 0)."""
+    x = _f32(logits)
+    if x.ndim == 1:
+        x = x[None, :]
+    rows, vocab = x.shape
+    out = np.zeros(rows, dtype=np.int32)
+    _load().oracle_argmax(rows, vocab, x, vocab, out)
+    return out
+
+
+def tree_accept(parent, token, target):
+    """Greedy acceptance of one tree: (path [T] root-first, -1 padded; len; bonus)."""
+    p = np.ascontiguousarray(parent, dtype=np.int32)
+    T = int(p.shape[0])
+    tok = np.ascontiguousarray(token, dtype=np.int32)
+    tgt = np.ascontiguousarray(target, dtype=np.int32)
+    assert tok.shape == (T,) and tgt.shape == (T,)
+    path = np.zeros(T, dtype=np.int32)
+    n = ctypes.c_int32(0)
+    bonus = ctypes.c_int32(0)
+    rc = _load().oracle_tree_accept(T, p, tok, tgt, path, ctypes.byref(n), ctypes.byref(bonus))
+    if rc != 0:
+        raise ValueError("malformed parent[]")
+    return path, int(n.value), int(bonus.value)
+
+
+def accept_commit(page_table, L: int, path, n: int) -> np.ndarray:
+    """Page table of one request ([L+T] slots) after committing the accepted path."""
+    pt = np.array(page_table, dtype=np.int32, copy=True)
+    pa = np.ascontiguousarray(path, dtype=np.int32)
+    T = int(pt.shape[0]) - int(L)
+    _load().oracle_accept_commit(int(L), T, int(n), pa, pt)
+    return pt
+
+
+def accept_case(case):
+    """Oracle acceptance of a whole ``datagen.AcceptCase``.
+
+    Returns dict with target [sumT], path [B][max_T] (-1 padded), len [B],
+    bonus [B], and page_table (committed copy) when the case has one.
+    """
+    target = argmax(case.logits) if case.logits is not None else np.asarray(case.target_in,
+                                                                            dtype=np.int32)
+    B = case.batch
+    path = np.full((B, case.max_T), -1, dtype=np.int32)
+    lens = np.zeros(B, dtype=np.int32)
+    bonus = np.zeros(B, dtype=np.int32)
+    pt = None if case.page_table is None else np.array(case.page_table, dtype=np.int32)
+    for b in range(B):
+        t0, t1 = int(case.tree_off[b]), int(case.tree_off[b + 1])
+        pb, n, bo = tree_accept(case.parent[t0:t1], case.token[t0:t1], target[t0:t1])
+        path[b, :t1 - t0] = pb
+        lens[b] = n
+        bonus[b] = bo
+        if pt is not None:
+            k0, k1 = int(case.kv_off[b]), int(case.kv_off[b + 1])
+            pt[k0:k1] = accept_commit(pt[k0:k1], int(case.prefix_len[b]), pb, n)
+    out = {"target": target, "path": path, "len": lens, "bonus": bonus}
+    if pt is not None:
+        out["page_table"] = pt
+    return out

@@ -290,4 +290,87 @@ void oracle_combine(int32_t S, int64_t rows, int32_t d, const double* o_part,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Greedy tree acceptance: the step after verification, which keeps the longest
+// run of draft tokens that the target model agrees with (page "The
+// Architecture of Diagnosis", section "Phase 1: Custom CUDA Kernels", item 3:
+// a device-side kernel picks the longest accepted prefix after verification).
+// The page gives no formula; the reading used here:
+//
+//   target[t] = argmax_v logits[t][v]: the lowest v among equal maxima; NaN
+//               entries never win; a row that is all NaN (or empty) gives 0.
+//   accepted  : a root (parent -1) is accepted; node u with parent p is
+//               accepted iff p is accepted and token[u] == target[p].
+//   end       : the accepted node of greatest depth, the lowest index among
+//               equal depths.
+//   path      : end's ancestor chain, root first; len = depth(end) + 1.
+//   bonus     : target[end], the target's own next token after the path.
+//   commit    : (page-table KV) logical key L+i of the request becomes the slot
+//               of path[i], for i < len -- the accepted nodes' KV rows move
+//               to the front of the tree region without copying any row; the
+//               other nodes' slots follow in node order.
+
+// target[r] for `rows` rows of `vocab` values (row stride ld). The values are
+// float32 storage (bf16 values are exact in it); plain comparisons decide.
+void oracle_argmax(int64_t rows, int64_t vocab, const float* logits, int64_t ld,
+                   int32_t* target) {
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* x = logits + r * ld;
+    int64_t best = -1;
+    for (int64_t v = 0; v < vocab; ++v) {
+      if (std::isnan(x[v])) continue;
+      if (best < 0 || x[v] > x[best]) best = v;   // strict: equal values keep the lower v
+    }
+    target[r] = (int32_t)(best < 0 ? 0 : best);
+  }
+}
+
+// Acceptance of ONE tree of T nodes. path must hold T entries; entries past
+// len are set to -1. Returns 0, or -1 when parent[] is not a discovery-ordered
+// forest (or T is not in [1, 64]).
+int oracle_tree_accept(int32_t T, const int32_t* parent, const int32_t* token,
+                       const int32_t* target, int32_t* path, int32_t* len, int32_t* bonus) {
+  if (T < 1 || T > 64) return -1;
+  std::vector<char> accepted(T, 0);
+  std::vector<int32_t> depth(T, 0);
+  for (int32_t u = 0; u < T; ++u) {
+    const int32_t p = parent[u];
+    if (p == -1) {
+      accepted[u] = 1;
+      depth[u] = 0;
+    } else if (p >= 0 && p < u) {
+      accepted[u] = accepted[p] && token[u] == target[p];
+      depth[u] = depth[p] + 1;
+    } else {
+      return -1;
+    }
+  }
+  int32_t end = -1;
+  for (int32_t u = 0; u < T; ++u)
+    if (accepted[u] && (end < 0 || depth[u] > depth[end])) end = u;
+  const int32_t n = depth[end] + 1;
+  for (int32_t i = 0; i < T; ++i) path[i] = -1;
+  for (int32_t u = end, i = n - 1; i >= 0; --i, u = parent[u]) path[i] = u;
+  *len = n;
+  *bonus = target[end];
+  return 0;
+}
+
+// Page-table commit of one request: pt is the request's logical->slot table
+// ([L+T] entries). The tree region [L, L+T) is reordered: first the slots of
+// the accepted path in path order, then the slots of the other nodes in node
+// order, so the table stays a permutation and the rejected nodes' slots end
+// up at [L+len, L+T) where the caller can recycle them.
+void oracle_accept_commit(int32_t L, int32_t T, int32_t len, const int32_t* path, int32_t* pt) {
+  std::vector<int32_t> old(pt + L, pt + L + T);
+  std::vector<char> on_path(T, 0);
+  int32_t k = 0;
+  for (int32_t i = 0; i < len; ++i) {
+    pt[L + k++] = old[path[i]];
+    on_path[path[i]] = 1;
+  }
+  for (int32_t u = 0; u < T; ++u)
+    if (!on_path[u]) pt[L + k++] = old[u];
+}
+
 }  // extern "C"

@@ -261,3 +261,132 @@ def scaled_case(case: VerifyCase, rows_scale: float) -> VerifyCase:
     if case.dtype == "bf16":
         q = bf16_round(q)
     return dataclasses.replace(case, q=q, name=f"{case.name}_qx{rows_scale}")
+
+
+# ---------------------------------------------------------------------------
+# Greedy tree acceptance inputs.
+#
+# The pages give no vocabulary size; the synthetic logits use 163,840 columns,
+# the vocabulary of the Kimi K2 tokenizer that the Kimi-shape layer belongs to.
+KIMI_VOCAB = 163_840
+
+
+@dataclasses.dataclass
+class AcceptCase:
+    """One batched greedy-acceptance problem.
+
+    ``logits`` rows are the target model's outputs at each tree node (node-major,
+    request after request); ``token[u]`` is the draft token of node u. Logical
+    key j of request b has slot ``page_table[kv_off[b] + j]`` (when paged).
+    """
+    name: str
+    vocab: int
+    max_T: int
+    parent: np.ndarray              # int32 [sumT]
+    tree_off: np.ndarray            # int32 [B+1]
+    token: np.ndarray               # int32 [sumT]
+    logits: Optional[np.ndarray]    # float32 [sumT, vocab] (bf16-exact when dtype bf16)
+    target_in: Optional[np.ndarray] # int32 [sumT] when logits is None
+    dtype: str                      # "bf16" or "f32"
+    prefix_len: np.ndarray          # int32 [B]
+    kv_off: np.ndarray              # int32 [B+1]
+    page_table: Optional[np.ndarray] = None
+    seed: int = 0
+
+    @property
+    def batch(self) -> int:
+        return int(self.tree_off.shape[0] - 1)
+
+    @property
+    def total_nodes(self) -> int:
+        return int(self.tree_off[-1])
+
+
+def make_accept_case(name: str, *, parents: List[np.ndarray], vocab: int, seed: int,
+                     p_follow: float = 0.8, dtype: str = "bf16", with_logits: bool = True,
+                     prefix_len: Optional[List[int]] = None, paged: bool = False,
+                     sibling_dups: bool = False, ties: bool = False,
+                     nan_rows: int = 0) -> AcceptCase:
+    """Draft tokens and target logits for a batch of trees.
+
+    Siblings get distinct tokens (unless ``sibling_dups``, which copies a
+    sibling's token now and then). At every node the planted target token is,
+    with probability ``p_follow``, the token of one of its children, else a
+    random token; the planted logit is 16.0, above every N(0,1) draw. ``ties``
+    plants the same 16.0 at a second random column; ``nan_rows`` rows get NaN
+    at random columns (one row entirely NaN when nan_rows > 0).
+    """
+    B = len(parents)
+    tree_T = np.array([len(p) for p in parents], dtype=np.int32)
+    tree_off = np.zeros(B + 1, dtype=np.int32)
+    tree_off[1:] = np.cumsum(tree_T)
+    sumT = int(tree_off[-1])
+    parent = np.concatenate([np.asarray(p, dtype=np.int32) for p in parents])
+    token = np.zeros(sumT, dtype=np.int32)
+    target = np.zeros(sumT, dtype=np.int32)
+    rt = rng_for(seed, "tokens")
+    for b in range(B):
+        t0, T = int(tree_off[b]), int(tree_T[b])
+        par = parent[t0:t0 + T]
+        token[t0] = int(rt.integers(0, vocab))
+        children = [[] for _ in range(T)]
+        for u in range(1, T):
+            if par[u] >= 0:
+                children[par[u]].append(u)
+        for p_ in range(T):
+            kids = children[p_]
+            if kids:
+                draw = rt.choice(vocab, size=len(kids), replace=False)
+                for k, u in enumerate(kids):
+                    token[t0 + u] = int(draw[k])
+                if sibling_dups and len(kids) > 1 and rt.random() < 0.5:
+                    token[t0 + kids[-1]] = token[t0 + kids[0]]
+            if kids and rt.random() < p_follow:
+                target[t0 + p_] = token[t0 + kids[int(rt.integers(0, len(kids)))]]
+            else:
+                target[t0 + p_] = int(rt.integers(0, vocab))
+    logits = None
+    if with_logits:
+        rl = rng_for(seed, "logits")
+        logits = rl.standard_normal((sumT, vocab), dtype=np.float32)
+        if dtype == "bf16":
+            logits = bf16_round(logits)
+        logits[np.arange(sumT), target] = 16.0
+        if ties:
+            logits[np.arange(sumT), rl.integers(0, vocab, size=sumT)] = 16.0
+        for i in range(min(nan_rows, sumT)):
+            r = int(rl.integers(0, sumT))
+            logits[r, rl.integers(0, vocab, size=16)] = np.nan
+        if nan_rows > 0:
+            logits[int(rl.integers(0, sumT))] = np.nan
+    if prefix_len is None:
+        prefix_len = [0] * B
+    plen = np.asarray(prefix_len, dtype=np.int32)
+    kv_off = np.zeros(B + 1, dtype=np.int32)
+    kv_off[1:] = np.cumsum(plen + tree_T)
+    page_table = None
+    if paged:
+        n_keys = int(kv_off[-1])
+        page_table = rng_for(seed, "perm", n_keys).permutation(n_keys).astype(np.int32)
+    return AcceptCase(name=name, vocab=vocab, max_T=int(tree_T.max()), parent=parent,
+                      tree_off=tree_off, token=token, logits=logits,
+                      target_in=None if with_logits else target, dtype=dtype,
+                      prefix_len=plen, kv_off=kv_off, page_table=page_table, seed=seed)
+
+
+def kimi_accept_case(T: int = 13, seed: int = 1, vocab: int = KIMI_VOCAB) -> AcceptCase:
+    """Acceptance after one Kimi-shape verify: one tree of T nodes (the same
+    tree draw as ``kimi_layer_case``), bf16 logits over the full vocabulary."""
+    parent = random_tree(T, rng_for(seed, "tree", T))
+    return make_accept_case(f"kimi_accept_T{T}", parents=[parent], vocab=vocab, seed=seed,
+                            prefix_len=[5553])
+
+
+def batched_accept_case(B: int = 8, seed: int = 4, vocab: int = KIMI_VOCAB) -> AcceptCase:
+    """Acceptance for the batched paged verify: the same prefixes, trees and
+    page-table permutation as ``batched_paged_case(B, seed=seed)``."""
+    plen = rng_for(seed, "prefix", B).integers(1024, 32768 + 1, size=B)
+    tT = rng_for(seed, "treeT", B).integers(9, 16 + 1, size=B)
+    parents = [random_tree(int(tT[b]), rng_for(seed, "tree", b, int(tT[b]))) for b in range(B)]
+    return make_accept_case(f"paged_accept_B{B}", parents=parents, vocab=vocab, seed=seed,
+                            prefix_len=[int(x) for x in plen], paged=True)
