@@ -38,6 +38,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <cstring>
+
 #include "kdv_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -67,7 +70,7 @@ constexpr int V_STAGES = 8;
 constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
 constexpr int NP = 2;
 constexpr int P_BYTES = ROWS * KEYS * 2;
-constexpr int P_KBLOCK_BYTES = ROWS * 128;
+constexpr int P_KCHUNK_BYTES = ROWS * 16;           // 8 keys of all 128 rows (interleaved core matrices)
 constexpr int P_MSG_BYTES = P_BYTES + ROWS * 4;
 constexpr int P_SLOT_BYTES = 33792;
 constexpr int STATS_BYTES = 2 * ROWS * 4;
@@ -175,7 +178,8 @@ __device__ __forceinline__ void arrive_on(uint32_t bar, uint32_t rank, uint32_t 
 
 __global__ void __launch_bounds__(THREADS, 1) __cluster_dims__(4, 1, 1)
 verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_v,
-                  const __grid_constant__ CUtensorMap tmap_q, const VerifyArgs a, const VerifyPlan p) {
+                  const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_o,
+                  const int o_tma, const VerifyArgs a, const VerifyPlan p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -445,10 +449,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             lsum += p0 + p1;
             w[q] = pack_bf16x2(p0, p1);
           }
-          const int kb = ch >> 3, piece = ch & 7;
-          if (ok)
-            st_async_v4(pslot + kb * P_KBLOCK_BYTES + r * 128 + ((piece ^ (r & 7)) << 4), w[0], w[1], w[2],
-                        w[3], pbar);
+          // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
+          // so a warp's 32 rows fill 512 contiguous bytes per store
+          if (ok) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, w[0], w[1], w[2], w[3], pbar);
         }
         l_part += lsum;
         // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
@@ -505,7 +508,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 #pragma unroll
           for (int kk = 0; kk < VKEYS / 16; ++kk) {
             const int k = (VKEYS / 16) * h + kk;
-            const uint64_t adesc = sw128_desc(pbuf + (k >> 2) * P_KBLOCK_BYTES + (k & 3) * 32, 16, 1024);
+            const uint64_t adesc = interleave_desc(pbuf + k * 2 * P_KCHUNK_BYTES, P_KCHUNK_BYTES, 128);
 #pragma unroll
             for (int nh = 0; nh < 2; ++nh) {
               // this CTA's 128 of the 256 columns: two 64-dim blocks, LBO apart
@@ -531,81 +534,117 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           mbar_arrive_remote_relaxed(peer_pempty + slot * 8);
         }
       }
-    } else if (warp >= WG_FIRST_WARP && warp < WG2_FIRST_WARP) {
-      // ---------------- rescale + epilogue (both O CTAs): thread <-> row
+    } else if (warp >= WG_FIRST_WARP) {
+      // ---------------- rescale (warps 4-7) and epilogue (warps 4-11), both
+      // O CTAs: thread <-> row; warpgroup eh stores columns [256*eh, 256*eh+256)
+      const int ew = warp - WG_FIRST_WARP;
+      const int eh = ew >> 2;
       const int sp = warp & 3;
       const int r = sp * 32 + lane;
       const int row = row0 + r;
       const bool valid = row < rows_b;
       const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-      bool ok = true;
-      for (int i = 0; i < n_ptiles; ++i) {
-        const int slot = i % NP;
-        ok = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1) && ok;
-        fence_proxy_async_smem();      // P arrived by st.async; the pair's MMA reads it
-        const float al = *reinterpret_cast<volatile float*>(smem + OFF_P + slot * P_SLOT_BYTES + P_BYTES + r * 4);
-        const bool need = ok && i > 0 && al != 1.f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O must be quiescent: wait for tile i-1's MMAs, then scale the rows
-          ok = wait_warp(c, c.bar(B_PV_DONE + (i - 1) % NP), ((i - 1) / NP) & 1) && ok;
-          if (__all_sync(0xffffffffu, ok)) {
-            __syncwarp();
-            tc_fence_after();
-            const float f = need ? al : 1.f;
+      bool bad = false;
+      if (eh == 0) {
+        bool ok = true;
+        for (int i = 0; i < n_ptiles; ++i) {
+          const int slot = i % NP;
+          ok = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1) && ok;
+          fence_proxy_async_smem();      // P arrived by st.async; the pair's MMA reads it
+          const float al = *reinterpret_cast<volatile float*>(smem + OFF_P + slot * P_SLOT_BYTES + P_BYTES + r * 4);
+          const bool need = ok && i > 0 && al != 1.f;
+          if (__any_sync(0xffffffffu, need)) {
+            // O must be quiescent: wait for tile i-1's MMAs, then scale the rows
+            ok = wait_warp(c, c.bar(B_PV_DONE + (i - 1) % NP), ((i - 1) / NP) & 1) && ok;
+            if (__all_sync(0xffffffffu, ok)) {
+              __syncwarp();
+              tc_fence_after();
+              const float f = need ? al : 1.f;
 #pragma unroll 1
-            for (int cb = 0; cb < DC / 32; ++cb) {
-              uint32_t v[32];
-              tmem_ld32(tmem + lane_base + cb * 32, v);
-              tmem_wait_ld();
+              for (int cb = 0; cb < DC / 32; ++cb) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + cb * 32, v);
+                tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
-              tmem_st32(tmem + lane_base + cb * 32, v);
+                for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * f);
+                tmem_st32(tmem + lane_base + cb * 32, v);
+              }
+              tmem_wait_st();
+              tc_fence_before();
             }
-            tmem_wait_st();
-            tc_fence_before();
           }
+          if (ok) arrive_on(c.bar(B_READY + slot), lead_rank, rank);
         }
-        if (ok) arrive_on(c.bar(B_READY + slot), lead_rank, rank);
+        // the final MMAs and the row statistics (waited in order: every
+        // earlier phase of these barriers is already known to be complete)
+        bool have_o = n_ptiles > 0;
+        if (have_o) {
+          const int i = n_ptiles - 1;
+          have_o = wait_warp(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
+        }
+        have_o = __all_sync(0xffffffffu, have_o);
+        ok = wait_warp(c, c.bar(B_STATS), 0) && ok && have_o == (n_ptiles > 0);
+        bad = !ok;
       }
-      // ---------------- epilogue: o = O / l, lse = ln2 * (m + log2 l)
-      bool have_o = n_ptiles > 0;
-      if (have_o) {
-        const int i = n_ptiles - 1;
-        have_o = wait_warp(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
-      }
-      have_o = __all_sync(0xffffffffu, have_o);
-      ok = wait_warp(c, c.bar(B_STATS), 0) && ok && have_o == (n_ptiles > 0);
-      __syncwarp();
+      // warps 8-11 learn of the final MMA and the statistics through this barrier
+      bad = named_bar_or(1, 2 * 128, bad);
+      const bool have_o = n_ptiles > 0 && !bad;
       tc_fence_after();
+      // ---------------- epilogue: o = O / l, lse = ln2 * (m + log2 l)
       const float l = *reinterpret_cast<volatile float*>(smem + OFF_STATS + r * 4);
       const float m = *reinterpret_cast<volatile float*>(smem + OFF_STATS + ROWS * 4 + r * 4);
-      const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
-      const float lse = (l > 0.f && ok) ? (m + __log2f(l)) * LN2 : -INFINITY;
+      const float inv = (l > 0.f && !bad) ? 1.f / l : 0.f;
+      const float lse = (l > 0.f && !bad) ? (m + __log2f(l)) * LN2 : -INFINITY;
       const int64_t orow = out_row_index(p, b, split, row);
+      // whole-warp rows go out as 32x32 fp32 boxes through the TMA store
+      // (staged 128B-swizzled in the V ring, free once the last PV is done);
+      // a warp straddling the end of the request stores row by row
+      const int wrow0 = row0 + sp * 32;
+      const bool warp_full = o_tma != 0 && !bad && wrow0 + 32 <= rows_b;
+      const int64_t wy = out_row_index(p, b, split, wrow0);
+      const uint32_t stage = base + OFF_RING + ew * 8192;
       float* orow_ptr = a.o + orow * DC;
 #pragma unroll 1
-      for (int cb = 0; cb < DC / 32; ++cb) {
+      for (int cb = 0; cb < 256 / 32; ++cb) {
+        const int col = eh * 256 + cb * 32;
         uint32_t v[32];
         if (have_o) {
-          tmem_ld32(tmem + lane_base + cb * 32, v);
+          tmem_ld32(tmem + lane_base + col, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) v[k] = 0u;
         }
-        if (valid) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float4 f;
-            f.x = __uint_as_float(v[4 * k + 0]) * inv;
-            f.y = __uint_as_float(v[4 * k + 1]) * inv;
-            f.z = __uint_as_float(v[4 * k + 2]) * inv;
-            f.w = __uint_as_float(v[4 * k + 3]) * inv;
-            *reinterpret_cast<float4*>(orow_ptr + cb * 32 + 4 * k) = f;
+        for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * inv);
+        if (warp_full) {
+          const uint32_t buf = stage + (cb & 1) * 4096;
+          if (cb >= 2) {
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
           }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(buf + lane * 128 + ((q ^ (lane & 7)) << 4)), "r"(v[4 * q]), "r"(v[4 * q + 1]),
+                            "r"(v[4 * q + 2]), "r"(v[4 * q + 3]) : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_o, buf, col, (int32_t)wy);
+            bulk_commit_group();
+          }
+        } else if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(orow_ptr + col + 4 * q) =
+                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
         }
       }
-      if (valid && a.lse != nullptr) a.lse[orow] = lse;
+      if (warp_full && lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
+      if (eh == 0 && valid && a.lse != nullptr) a.lse[orow] = lse;
     }
   }
 
@@ -652,11 +691,26 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   };
-  CUtensorMap tmap_kv, tmap_v, tmap_q;
+  CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o;
   if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, HKEYS) != CUDA_SUCCESS ||
       make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, VKEYS) != CUDA_SUCCESS ||
       make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  // output rows as fp32 [rows][512] for the epilogue's 32x32 TMA stores
+  int64_t out_rows = 0;
+  for (int b = 0; b < p.B; ++b)
+    if (p.T[b] > 0) out_rows = std::max<int64_t>(out_rows, out_row_index(p, b, p.S[b] - 1, p.T[b] * p.H - 1) + 1);
+  int o_tma = 0;
+  std::memset(&tmap_o, 0, sizeof(tmap_o));
+  if (out_rows > 0 && out_rows <= (int64_t)0x7fffffff && (reinterpret_cast<uintptr_t>(a.o) & 15) == 0) {
+    const cuuint64_t dims[2] = {(cuuint64_t)DC, (cuuint64_t)out_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)DC * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    o_tma = enc(&tmap_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.o, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS ? 1 : 0;
+  }
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -666,7 +720,7 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  verify_tc2_kernel<<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, a, p);
+  verify_tc2_kernel<<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
   return cudaGetLastError();
 }
 
