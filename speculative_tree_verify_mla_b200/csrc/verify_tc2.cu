@@ -209,6 +209,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   const int k_lo = min(split * p.chunk[b], n_keys);
   const int k_hi = min(k_lo + p.chunk[b], n_keys);
   const int n_stiles = (k_hi - k_lo + STILE - 1) / STILE;
+  auto stile_key = [&](int i) { return k_lo + i * STILE; };
   const int n_ptiles = 2 * n_stiles;
   const int64_t kv_base = a.kv_off[b];
 
@@ -221,11 +222,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         mbar_init(c.bar(B_KV_EMPTY + i), 1);
       }
       mbar_init(c.bar(B_S_FULL), 1);
-      mbar_init(c.bar(B_S_EMPTY), 4 * ROWS);             // both warpgroups of both S CTAs
+      mbar_init(c.bar(B_S_EMPTY), 16);                   // every softmax warp of both S CTAs
       for (int i = 0; i < NP; ++i) mbar_init(c.bar(B_P_EMPTY + i), 1);
       mbar_init(c.bar(B_QLAT_FULL), 1);
       mbar_init(c.bar(B_QROPE_FULL), 1);
-      mbar_init(c.bar(B_Q_READY), 2 * ROWS);
+      mbar_init(c.bar(B_Q_READY), 8);                    // the q_lat-copying warps of both S CTAs
       mbar_init(c.bar(B_S_DRAIN), 1);
       // KV_FULL phase k of ring stage st belongs to ring use st + 4k; the
       // stages that hold q_lat at start-up (uses 0-2) carry no KV, so their
@@ -245,7 +246,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       }
       for (int i = 0; i < NP; ++i) {
         mbar_init(c.bar(B_P_FULL + i), 1);
-        mbar_init(c.bar(B_READY + i), 2 * ROWS);
+        mbar_init(c.bar(B_READY + i), 8);                // the rescale warps of both O CTAs
         mbar_init(c.bar(B_PV_DONE + i), 1);
       }
       mbar_init(c.bar(B_STATS), 1);
@@ -286,7 +287,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         if (!wait_bar(c, c.bar(B_KV_EMPTY + st), ((pos / KV_STAGES) & 1) ^ 1)) break;
         if (leader) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KV_STAGE_BYTES);
         const int tile = g / STAGES_PER_TILE, blk0 = (g % STAGES_PER_TILE) * STAGE_BLOCKS;
-        const int32_t y = (int32_t)(kv_base + k_lo + tile * STILE + (int)half * HKEYS);
+        const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
         const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
         for (int e = 0; e < STAGE_BLOCKS; ++e)
           tma_load_2d_pair(base + OFF_RING + st * KV_STAGE_BYTES + e * KBLOCK_BYTES, &tmap_kv, fb, (blk0 + e) * 64, y);
@@ -374,7 +375,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           tmem_wait_st();
         }
         tc_fence_before();
-        arrive_on(c.bar(B_Q_READY), lead_rank, rank);
+        __syncwarp();
+        if (lane == 0) arrive_on(c.bar(B_Q_READY), lead_rank, rank);
       }
       const uint64_t mask_t = valid ? a.mask[p.tree_base[b] + row / H] : 0ull;
       const float sl2 = a.scale * LOG2E;
@@ -396,13 +398,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
           tmem_wait_ld();
           tc_fence_before();
-          arrive_on(c.bar(B_S_EMPTY), lead_rank, rank);
+          __syncwarp();
+          if (lane == 0) arrive_on(c.bar(B_S_EMPTY), lead_rank, rank);
         } else {
 #pragma unroll
           for (int k = 0; k < KEYS; ++k) sv[k] = 0u;
         }
         ok = ok && wok;
-        const int key0 = k_lo + i * STILE + hw * KEYS;
+        const int key0 = stile_key(i) + hw * KEYS;
         float m_half = -INFINITY;
         if (valid && key0 + KEYS <= min(L, k_hi)) {
 #pragma unroll
@@ -481,7 +484,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const int st = u % V_STAGES;
         if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1)) break;
         if (leader) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
-        const int32_t y = (int32_t)(kv_base + k_lo + u * VKEYS);
+        const int32_t y = (int32_t)(kv_base + stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS);
         const uint32_t dst = base + OFF_RING + st * V_STAGE_BYTES;
         const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
         for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
@@ -573,7 +576,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
               tc_fence_before();
             }
           }
-          if (ok) arrive_on(c.bar(B_READY + slot), lead_rank, rank);
+          __syncwarp();
+          if (ok && lane == 0) arrive_on(c.bar(B_READY + slot), lead_rank, rank);
         }
         // the final MMAs and the row statistics (waited in order: every
         // earlier phase of these barriers is already known to be complete)
