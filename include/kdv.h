@@ -210,6 +210,70 @@ KDV_API kdv_status kdv_verify_attn_noalloc(const kdv_verify_params* p, void* str
 KDV_API kdv_status kdv_combine(const float* o_part, const float* lse_part, int32_t S, int64_t rows,
                        int32_t d, float* o, float* lse, void* stream);
 
+/*
+ * Greedy tree acceptance -- the step after verification: keep the longest
+ * run of draft tokens that the target model agrees with (page "The
+ * Architecture of Diagnosis", section "Phase 1: Custom CUDA Kernels", item 3:
+ * a device-side kernel selects the longest accepted prefix with no host
+ * involvement). The page gives no formula; this library reads it as:
+ *   target[t] = argmax_v logits[t][v]: the lowest v among equal maxima, NaN
+ *               never wins, a row of only NaN gives 0. (Or taken as given
+ *               from target_in when logits is NULL.)
+ *   accepted  : a root (parent -1) is accepted; node u with parent p is
+ *               accepted iff p is accepted and token[u] == target[p].
+ *   end       : the accepted node of greatest depth (lowest index on ties);
+ *   path      : end's ancestor chain, root first; accept_len = depth(end)+1;
+ *   bonus     : target[end], the target model's next token after the path.
+ * Page commit (optional, page_size = 1): the tree region [L, L+T) of the
+ * request's page table is reordered in place so that logical key L+i holds
+ * the slot of path[i] (i < accept_len) and the other nodes' slots follow in
+ * node order -- the accepted KV rows move to the front without copying a row
+ * (the non-contiguous KV commit of page "The Architecture of Diagnosis",
+ * section "The Discrepancy That Revealed the Truth", item 2), and the
+ * rejected nodes' slots end up at [L+accept_len, L+T) for reuse.
+ */
+typedef struct kdv_accept_params {
+  int32_t batch;          /* B in [1, KDV_MAX_BATCH]                              */
+  int32_t max_T;          /* [1, 64]: bound on every T_b, row stride of path     */
+  int32_t total_nodes;    /* sumT = tree_off[B] (HOST value; rows of logits)     */
+  int32_t vocab;          /* V >= 1: logits columns; tokens lie in [0, V)        */
+  int32_t dtype;          /* KDV_BF16 or KDV_F32: element type of logits         */
+  const void* logits;     /* [sumT][logits_ld] target logits, or NULL            */
+  int64_t logits_ld;      /* elements between logits rows (>= vocab)             */
+  const int32_t* target_in;   /* [sumT] target tokens, read when logits is NULL  */
+  const int32_t* token;       /* [sumT] draft token of each node (roots: unused) */
+  const int32_t* parent;      /* [sumT] local parent, -1 for a root              */
+  const int32_t* tree_off;    /* [B+1] device CSR offsets                        */
+  int32_t* target_out;        /* [sumT] out, nullable: target[t]                 */
+  int32_t* accept_len;        /* [B] out: accepted nodes, root included          */
+  int32_t* accept_path;       /* [B][max_T] out: local node ids root first, -1 pad */
+  int32_t* bonus;             /* [B] out, nullable: target at the path's end     */
+  int32_t* page_table;        /* nullable: [kv_off[B]] slots, committed in place */
+  const int32_t* kv_off;      /* [B+1] device, required with page_table          */
+  const int32_t* prefix_len;  /* [B] device, required with page_table or prefix_len_out */
+  int32_t* prefix_len_out;    /* [B] out, nullable: prefix_len + accept_len (may
+                                 be the prefix_len array itself)                 */
+  void* workspace;            /* caller scratch, >= kdv_tree_accept_workspace    */
+  size_t workspace_bytes;
+  int32_t* d_err;             /* nullable device error flag                      */
+} kdv_accept_params;
+
+/* Bytes of workspace kdv_tree_accept needs (0 when logits is NULL). */
+KDV_API kdv_status kdv_tree_accept_workspace(const kdv_accept_params* p, size_t* bytes);
+
+/*
+ * kdv_tree_accept -- argmax of the target logits at every node, greedy path
+ * selection, and the optional page-table commit, all on the device.
+ * Requirements: logits 16-byte aligned and logits_ld*elem a multiple of 16
+ * bytes for the vector path (other layouts take a scalar path). Device-side
+ * errors: KDV_DERR_BAD_PARENT (that request gets accept_len 0, path -1,
+ * bonus -1, no commit), KDV_DERR_BAD_TOKEN (a draft or given target token
+ * outside [0, V); it is compared as is), KDV_DERR_BAD_LENGTH (T_b outside
+ * [1, max_T], or the page-table range of a request shorter than L_b + T_b:
+ * no commit for that request).
+ */
+KDV_API kdv_status kdv_tree_accept(const kdv_accept_params* p, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

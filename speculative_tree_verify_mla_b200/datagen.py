@@ -309,8 +309,8 @@ def make_accept_case(name: str, *, parents: List[np.ndarray], vocab: int, seed: 
                      nan_rows: int = 0) -> AcceptCase:
     """Draft tokens and target logits for a batch of trees.
 
-    Siblings get distinct tokens (unless ``sibling_dups``, which copies a
-    sibling's token now and then). At every node the planted target token is,
+    Siblings get distinct tokens while the vocabulary allows it (and unless
+    ``sibling_dups``, which copies a sibling's token now and then). At every node the planted target token is,
     with probability ``p_follow``, the token of one of its children, else a
     random token; the planted logit is 16.0, above every N(0,1) draw. ``ties``
     plants the same 16.0 at a second random column; ``nan_rows`` rows get NaN
@@ -336,7 +336,7 @@ def make_accept_case(name: str, *, parents: List[np.ndarray], vocab: int, seed: 
         for p_ in range(T):
             kids = children[p_]
             if kids:
-                draw = rt.choice(vocab, size=len(kids), replace=False)
+                draw = rt.choice(vocab, size=len(kids), replace=len(kids) > vocab)
                 for k, u in enumerate(kids):
                     token[t0 + u] = int(draw[k])
                 if sibling_dups and len(kids) > 1 and rt.random() < 0.5:

@@ -42,7 +42,8 @@ KDV_MAX_BATCH = 128
 # Every entry point include/kdv.h declares (checked by the CPU tests).
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
-            "kdv_verify_attn_noalloc", "kdv_combine")
+            "kdv_verify_attn_noalloc", "kdv_combine", "kdv_tree_accept_workspace",
+            "kdv_tree_accept")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -68,6 +69,23 @@ class VerifyParams(ctypes.Structure):
         ("return_partials", ctypes.c_int32),
         ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("o_part", ctypes.c_void_p), ("lse_part", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("d_err", ctypes.c_void_p),
+    ]
+
+
+class AcceptParams(ctypes.Structure):
+    """Mirror of ``kdv_accept_params`` (field order and types must match kdv.h)."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("max_T", ctypes.c_int32),
+        ("total_nodes", ctypes.c_int32), ("vocab", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("logits", ctypes.c_void_p), ("logits_ld", ctypes.c_int64),
+        ("target_in", ctypes.c_void_p), ("token", ctypes.c_void_p),
+        ("parent", ctypes.c_void_p), ("tree_off", ctypes.c_void_p),
+        ("target_out", ctypes.c_void_p), ("accept_len", ctypes.c_void_p),
+        ("accept_path", ctypes.c_void_p), ("bonus", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p), ("kv_off", ctypes.c_void_p),
+        ("prefix_len", ctypes.c_void_p), ("prefix_len_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("d_err", ctypes.c_void_p),
     ]
@@ -103,6 +121,10 @@ def load() -> ctypes.CDLL:
         lib.kdv_combine.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int64, c.c_int32,
                                     c.c_void_p, c.c_void_p, c.c_void_p]
         lib.kdv_combine.restype = c.c_int
+        lib.kdv_tree_accept_workspace.argtypes = [c.POINTER(AcceptParams), c.POINTER(c.c_size_t)]
+        lib.kdv_tree_accept_workspace.restype = c.c_int
+        lib.kdv_tree_accept.argtypes = [c.POINTER(AcceptParams), c.c_void_p]
+        lib.kdv_tree_accept.restype = c.c_int
         _lib = lib
     return _lib
 
@@ -272,6 +294,96 @@ class DeviceCase:
         if self.return_partials:
             return self.o_part.cpu().numpy(), self.lse_part.cpu().numpy()
         return self.o.cpu().numpy(), self.lse.cpu().numpy()
+
+    def error_flag(self) -> int:
+        torch.cuda.synchronize()
+        return int(self.d_err.item())
+
+
+# ---------------------------------------------------------------------------
+# Greedy tree acceptance.
+# ---------------------------------------------------------------------------
+def make_accept_params(**kw) -> AcceptParams:
+    """Build an AcceptParams from keyword arguments (tensors become pointers)."""
+    p = AcceptParams()
+    for k, v in kw.items():
+        if isinstance(v, torch.Tensor):
+            setattr(p, k, int(v.data_ptr()))
+        else:
+            setattr(p, k, v)
+    return p
+
+
+def kdv_tree_accept_workspace(params: AcceptParams) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().kdv_tree_accept_workspace(ctypes.byref(params), ctypes.byref(n)),
+           "kdv_tree_accept_workspace")
+    return int(n.value)
+
+
+def kdv_tree_accept(params: AcceptParams, stream=None) -> None:
+    _check(load().kdv_tree_accept(ctypes.byref(params), _stream(stream)), "kdv_tree_accept")
+
+
+class DeviceAcceptCase:
+    """A ``datagen.AcceptCase`` uploaded to the GPU, plus output buffers.
+
+    ``run()`` calls kdv_tree_accept through the C ABI; the page table (when
+    the case has one) is committed in place, so ``run()`` restores it first.
+    """
+
+    def __init__(self, case, device="cuda", commit: bool = True, update_prefix: bool = True):
+        dev = torch.device(device)
+        self.case = case
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        self.logits = None
+        self.dtype = KDV_BF16 if case.dtype == "bf16" else KDV_F32
+        if case.logits is not None:
+            tdt = torch.bfloat16 if case.dtype == "bf16" else torch.float32
+            self.logits = torch.from_numpy(case.logits).to(tdt).to(dev)
+        self.target_in = i32(case.target_in) if case.target_in is not None else None
+        self.token = i32(case.token)
+        self.parent = i32(case.parent)
+        self.tree_off = i32(case.tree_off)
+        self.kv_off = i32(case.kv_off)
+        self.prefix_len = i32(case.prefix_len)
+        self.page_table0 = i32(case.page_table) if (case.page_table is not None and commit) else None
+        self.page_table = self.page_table0.clone() if self.page_table0 is not None else None
+        sumT, B = case.total_nodes, case.batch
+        self.target_out = torch.full((sumT,), -7, dtype=torch.int32, device=dev)
+        self.accept_len = torch.full((B,), -7, dtype=torch.int32, device=dev)
+        self.accept_path = torch.full((B, case.max_T), -7, dtype=torch.int32, device=dev)
+        self.bonus = torch.full((B,), -7, dtype=torch.int32, device=dev)
+        self.prefix_len_out = torch.full((B,), -7, dtype=torch.int32, device=dev) if update_prefix else None
+        self.d_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.params = make_accept_params(
+            batch=B, max_T=case.max_T, total_nodes=sumT, vocab=case.vocab, dtype=self.dtype,
+            logits=self.logits, logits_ld=case.vocab, target_in=self.target_in, token=self.token,
+            parent=self.parent, tree_off=self.tree_off, target_out=self.target_out,
+            accept_len=self.accept_len, accept_path=self.accept_path, bonus=self.bonus,
+            page_table=self.page_table, kv_off=self.kv_off, prefix_len=self.prefix_len,
+            prefix_len_out=self.prefix_len_out, workspace=None, workspace_bytes=0,
+            d_err=self.d_err)
+        self.ws_bytes = kdv_tree_accept_workspace(self.params)
+        self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.params.workspace = int(self.workspace.data_ptr())
+        self.params.workspace_bytes = self.ws_bytes
+
+    def run(self, stream=None):
+        if self.page_table is not None:
+            self.page_table.copy_(self.page_table0)
+        kdv_tree_accept(self.params, stream)
+        return self
+
+    def results(self) -> dict:
+        torch.cuda.synchronize()
+        out = {"target": self.target_out.cpu().numpy(), "path": self.accept_path.cpu().numpy(),
+               "len": self.accept_len.cpu().numpy(), "bonus": self.bonus.cpu().numpy()}
+        if self.page_table is not None:
+            out["page_table"] = self.page_table.cpu().numpy()
+        if self.prefix_len_out is not None:
+            out["prefix_len_out"] = self.prefix_len_out.cpu().numpy()
+        return out
 
     def error_flag(self) -> int:
         torch.cuda.synchronize()

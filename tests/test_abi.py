@@ -41,18 +41,20 @@ def test_status_strings(lib):
     assert kdv.kdv_version() == 100
 
 
-def test_params_struct_layout(tmp_path):
+@pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
+                                       (kdv.AcceptParams, "kdv_accept_params")])
+def test_params_struct_layout(tmp_path, cls, cname):
     """ctypes mirror matches the C struct: compile a probe against kdv.h."""
-    fields = [f[0] for f in kdv.VerifyParams._fields_]
+    fields = [f[0] for f in cls._fields_]
     src = tmp_path / "probe.c"
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "kdv.h"\nint main(void){'
-                   + "".join(f'printf("%zu\\n", offsetof(kdv_verify_params, {f}));' for f in fields)
-                   + 'printf("%zu\\n", sizeof(kdv_verify_params)); return 0;}')
+                   + "".join(f'printf("%zu\\n", offsetof({cname}, {f}));' for f in fields)
+                   + f'printf("%zu\\n", sizeof({cname})); return 0;}}')
     exe = tmp_path / "probe"
     import subprocess
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(x) for x in subprocess.check_output([str(exe)]).split()]
-    want = [getattr(kdv.VerifyParams, f).offset for f in fields] + [ctypes.sizeof(kdv.VerifyParams)]
+    want = [getattr(cls, f).offset for f in fields] + [ctypes.sizeof(cls)]
     assert got == want
 
 
@@ -129,6 +131,47 @@ def test_combine_validation(lib):
     assert f(None, None, 0, 4, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
     assert f(None, None, 2, 4, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
     assert f(None, None, 2, -1, 8, None, None, None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def _accept(**over):
+    base = dict(batch=2, max_T=8, total_nodes=10, vocab=1000, dtype=kdv.KDV_BF16, logits=0x1000,
+                logits_ld=1000, target_in=None, token=0x2000, parent=0x3000, tree_off=0x4000,
+                target_out=None, accept_len=0x5000, accept_path=0x6000, bonus=None,
+                page_table=None, kv_off=None, prefix_len=None, prefix_len_out=None,
+                workspace=None, workspace_bytes=0, d_err=None)
+    base.update(over)
+    return kdv.make_accept_params(**base)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(batch=0), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(batch=129, total_nodes=129), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(max_T=65), kdv.KDV_ERR_UNSUPPORTED),
+    (dict(total_nodes=17), kdv.KDV_ERR_INVALID_ARG),          # > batch * max_T
+    (dict(total_nodes=1), kdv.KDV_ERR_INVALID_ARG),           # < batch
+    (dict(vocab=0), kdv.KDV_ERR_INVALID_ARG),
+    (dict(dtype=5), kdv.KDV_ERR_INVALID_ARG),
+    (dict(logits_ld=999), kdv.KDV_ERR_INVALID_ARG),
+    (dict(logits=None), kdv.KDV_ERR_INVALID_ARG),             # neither logits nor target_in
+    (dict(token=None), kdv.KDV_ERR_INVALID_ARG),
+    (dict(accept_path=None), kdv.KDV_ERR_INVALID_ARG),
+    (dict(page_table=0x7000), kdv.KDV_ERR_INVALID_ARG),       # no kv_off / prefix_len
+    (dict(prefix_len_out=0x7000), kdv.KDV_ERR_INVALID_ARG),   # no prefix_len
+])
+def test_accept_host_validation(lib, over, status):
+    p = _accept(**over)
+    n = ctypes.c_size_t(0)
+    assert lib.kdv_tree_accept_workspace(ctypes.byref(p), ctypes.byref(n)) == status
+    assert lib.kdv_tree_accept(ctypes.byref(p), None) == status
+
+
+def test_accept_workspace(lib):
+    # one 64-bit key per (node, 8192-logit chunk)
+    assert kdv.kdv_tree_accept_workspace(_accept()) == 10 * 1 * 8
+    assert kdv.kdv_tree_accept_workspace(_accept(vocab=163840, logits_ld=163840)) == 10 * 20 * 8
+    assert kdv.kdv_tree_accept_workspace(_accept(logits=None, target_in=0x1000)) == 0
+    # a missing workspace is refused before any launch
+    assert lib.kdv_tree_accept(ctypes.byref(_accept()), None) == kdv.KDV_ERR_WORKSPACE
 
 
 def test_library_has_no_oracle_dependency():
