@@ -72,9 +72,10 @@ typedef enum {
 #define KDV_F32 1
 
 /* Kernel family for kdv_verify_attn. AUTO picks the tensor-core kernel when
- * its shape constraints hold (bf16, d_latent=512, d_rope=64, no page table),
- * else SIMT. TC runs 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per
- * work item); TC_1SM is the 1-SM-MMA variant (2-CTA clusters, 128 rows). */
+ * its shape constraints hold (bf16, d_latent=512, d_rope=64), else SIMT. TC
+ * runs 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per work item) and
+ * reads a paged pool with TMA four-row gathers; TC_1SM is the 1-SM-MMA
+ * variant (2-CTA clusters, 128 rows, contiguous KV only). */
 #define KDV_IMPL_AUTO 0
 #define KDV_IMPL_SIMT 1
 #define KDV_IMPL_TC 2

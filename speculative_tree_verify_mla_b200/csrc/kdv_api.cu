@@ -32,7 +32,7 @@ bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_1SM; }
 
 int resolve_impl(const kdv_verify_params* p) {
   if (p->impl == KDV_IMPL_SIMT || is_tc(p->impl)) return p->impl;
-  return (tc_shape_ok(p) && p->page_table == nullptr) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
+  return tc_shape_ok(p) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
 }
 
 // Host-side checks that need no device access.
@@ -56,7 +56,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->return_partials && p->num_splits < 1) return KDV_ERR_INVALID_ARG;
   if (is_tc(impl)) {
     if (!tc_shape_ok(p)) return KDV_ERR_UNSUPPORTED;
-    if (p->page_table != nullptr) return KDV_ERR_UNSUPPORTED;
+    if (p->page_table != nullptr && impl == KDV_IMPL_TC_1SM) return KDV_ERR_UNSUPPORTED;
   } else {
     if (p->d_latent > 512 || p->d_rope > 64) return KDV_ERR_UNSUPPORTED;
   }

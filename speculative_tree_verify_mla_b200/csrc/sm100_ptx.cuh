@@ -187,6 +187,14 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap,
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
       :: "r"(dst), "l"(tmap), "r"(cluster_bar), "r"(x), "r"(y) : "memory");
 }
+// Four-row gather, pair form: like tma_load_2d_pair, completing on the
+// leader CTA's barrier; the tensor map's box is one row high.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const void* tmap, uint32_t cluster_bar, int32_t x,
+                                                 int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      :: "r"(dst), "l"(tmap), "r"(cluster_bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" :: "r"(cluster_bar), "r"(bytes) : "memory");
 }

@@ -176,6 +176,21 @@ __device__ __forceinline__ void arrive_on(uint32_t bar, uint32_t rank, uint32_t 
   else mbar_arrive_remote_relaxed(mapa(bar, rank));
 }
 
+// Pool row of logical key j (paged KV, page_size 1). Keys past the split's
+// end (the tail of a partial tile, masked out by the softmax) reuse the last
+// key's row, so every row read is one the caller handed in; a slot outside
+// [0, num_slots) is reported and replaced by row 0.
+__device__ __forceinline__ int32_t paged_slot(const VerifyArgs& a, int64_t kv_base, int j, int k_hi) {
+  const int jj = j < k_hi ? j : k_hi - 1;
+  int32_t s = a.page_table[kv_base + jj];
+  if (s < 0 || (int64_t)s >= a.num_slots) {
+    record_error(a.d_err, KDV_DERR_BAD_SLOT);
+    s = 0;
+  }
+  return s;
+}
+
+template <bool PAGED>
 __global__ void __launch_bounds__(THREADS, 1) __cluster_dims__(4, 1, 1)
 verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_v,
                   const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_o,
@@ -269,12 +284,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 
   if (s_side) {
     // ======================================================= S pair
-    if (warp == 0 && lane == 0) {
+    if (warp == 0 && (PAGED || lane == 0)) {
       // ---------------- producer (both S CTAs): q_lat staging (local), q_rope
-      // and this CTA's 128 of every 256 KV rows (counted on the leader's barriers)
+      // and this CTA's 128 of every 256 KV rows (counted on the leader's
+      // barriers). Paged KV: the whole warp gathers, 4 rows per lane.
       const int n_stg = n_stiles * STAGES_PER_TILE;
       int issued = 0;
-      if (n_stiles > 0) {
+      int32_t slot[4] = {0, 0, 0, 0};
+      if (n_stiles > 0 && lane == 0) {
         const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
         mbar_arrive_expect_tx(c.bar(B_QLAT_FULL), QLAT_BLOCKS * QBLOCK_BYTES);
         for (int blk = 0; blk < QLAT_BLOCKS; ++blk)
@@ -284,17 +301,31 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       }
       for (int g = 0; g < n_stg; ++g) {
         const int pos = g + Q_STAGES, st = pos % KV_STAGES;
-        if (!wait_bar(c, c.bar(B_KV_EMPTY + st), ((pos / KV_STAGES) & 1) ^ 1)) break;
-        if (leader) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KV_STAGE_BYTES);
+        const uint32_t eparity = ((pos / KV_STAGES) & 1) ^ 1;
+        if (!(PAGED ? wait_warp(c, c.bar(B_KV_EMPTY + st), eparity) : wait_bar(c, c.bar(B_KV_EMPTY + st), eparity)))
+          break;
+        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KV_STAGE_BYTES);
         const int tile = g / STAGES_PER_TILE, blk0 = (g % STAGES_PER_TILE) * STAGE_BLOCKS;
-        const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
         const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
-        for (int e = 0; e < STAGE_BLOCKS; ++e)
-          tma_load_2d_pair(base + OFF_RING + st * KV_STAGE_BYTES + e * KBLOCK_BYTES, &tmap_kv, fb, (blk0 + e) * 64, y);
+        const uint32_t dst = base + OFF_RING + st * KV_STAGE_BYTES;
+        if (PAGED) {
+          if (g % STAGES_PER_TILE == 0) {
+            const int j0 = stile_key(tile) + (int)half * HKEYS + 4 * lane;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) slot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
+          }
+          for (int e = 0; e < STAGE_BLOCKS; ++e)
+            tma_gather4_pair(dst + e * KBLOCK_BYTES + lane * 512, &tmap_kv, fb, (blk0 + e) * 64, slot[0], slot[1],
+                             slot[2], slot[3]);
+        } else {
+          const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
+          for (int e = 0; e < STAGE_BLOCKS; ++e)
+            tma_load_2d_pair(dst + e * KBLOCK_BYTES, &tmap_kv, fb, (blk0 + e) * 64, y);
+        }
         issued = g + 1;
       }
-      if (n_stiles > 0) wait_bar(c, c.bar(B_QLAT_FULL), 0, true);
-      if (leader) {
+      if (n_stiles > 0 && lane == 0) wait_bar(c, c.bar(B_QLAT_FULL), 0, true);
+      if (leader && lane == 0) {
         // retire copies in flight (both halves count on the leader's barriers)
         if (n_stiles > 0) wait_bar(c, c.bar(B_QROPE_FULL), 0, true);
         for (int g = max(0, issued - KV_STAGES); g < issued; ++g) {
@@ -475,25 +506,43 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
     }
   } else {
     // ======================================================= O pair
-    if (warp == 0 && lane == 0) {
+    if (warp == 0 && (PAGED || lane == 0)) {
       // ---------------- V producer (both O CTAs): this CTA's 256 dims of
-      // every 32 keys; local block lb holds dims 64*((lb/2)*4 + half*2 + lb%2)
+      // every 32 keys; local block lb holds dims 64*((lb/2)*4 + half*2 + lb%2).
+      // Paged KV: lanes 0-7 gather 4 rows each.
       int issued = 0;
       const int n_sub = (KEYS / VKEYS) * n_ptiles;
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
-        if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1)) break;
-        if (leader) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
-        const int32_t y = (int32_t)(kv_base + stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS);
+        const uint32_t eparity = ((u / V_STAGES) & 1) ^ 1;
+        if (!(PAGED ? wait_warp(c, c.bar(B_V_EMPTY + st), eparity) : wait_bar(c, c.bar(B_V_EMPTY + st), eparity)))
+          break;
+        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
+        const int key0 = stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS;
         const uint32_t dst = base + OFF_RING + st * V_STAGE_BYTES;
         const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
-        for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
-          const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-          tma_load_2d_pair(dst + lb * VBLOCK_BYTES, &tmap_v, fb, gb * 64, y);
+        if (PAGED) {
+          if (lane < VKEYS / 4) {
+            int32_t slot[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) slot[q] = paged_slot(a, kv_base, key0 + 4 * lane + q, k_hi);
+            for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
+              const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
+              tma_gather4_pair(dst + lb * VBLOCK_BYTES + lane * 512, &tmap_v, fb, gb * 64, slot[0], slot[1], slot[2],
+                               slot[3]);
+            }
+          }
+          __syncwarp();
+        } else {
+          const int32_t y = (int32_t)(kv_base + key0);
+          for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
+            const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
+            tma_load_2d_pair(dst + lb * VBLOCK_BYTES, &tmap_v, fb, gb * 64, y);
+          }
         }
         issued = u + 1;
       }
-      if (leader)
+      if (leader && lane == 0)
         for (int u = max(0, issued - V_STAGES); u < issued; ++u)
           wait_bar(c, c.bar(B_V_FULL + u % V_STAGES), (u / V_STAGES) & 1, true);
     } else if (warp == 1 && lane == 0 && leader) {
@@ -696,8 +745,10 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   };
   CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o;
-  if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, HKEYS) != CUDA_SUCCESS ||
-      make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, VKEYS) != CUDA_SUCCESS ||
+  const bool paged = a.page_table != nullptr;
+  // paged KV: one map with one-row boxes serves the K and V gathers
+  if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : HKEYS) != CUDA_SUCCESS ||
+      make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : VKEYS) != CUDA_SUCCESS ||
       make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // output rows as fp32 [rows][512] for the epilogue's 32x32 TMA stores
@@ -720,11 +771,16 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(verify_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    e = cudaFuncSetAttribute(verify_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(verify_tc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  verify_tc2_kernel<<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
+  if (paged)
+    verify_tc2_kernel<true><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
+  else
+    verify_tc2_kernel<false><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
   return cudaGetLastError();
 }
 
@@ -733,7 +789,7 @@ int tc2_max_active_clusters() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
   if (cached[dev] > 0) return cached[dev];
-  if (cudaFuncSetAttribute(verify_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+  if (cudaFuncSetAttribute(verify_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -749,7 +805,7 @@ int tc2_max_active_clusters() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, verify_tc2_kernel, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
+  if (cudaOccupancyMaxActiveClusters(&n, verify_tc2_kernel<false>, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
   cached[dev] = n;
   return n;
 }

@@ -89,3 +89,63 @@ def test_tc_matches_simt_on_same_inputs(impl):
     o1, l1 = _run(case, impl, splits=2)
     o2, l2 = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_SIMT, num_splits=2).run().results()
     assert_parity(o1, l1, o2, l2)
+
+
+# ---------------------------------------------------------------------------
+# Paged KV (page_size 1) on the 2-SM kernel: TMA four-row gathers through the
+# page table.
+
+def test_tc_paged_bit_identical_to_contiguous():
+    """A random-permutation page table over a permuted pool gives exactly the
+    output of the identity layout (same logical key order, same arithmetic)."""
+    parents = [datagen.random_tree(T, np.random.default_rng(T + 3)) for T in (13, 9, 16)]
+    kw = dict(**datagen.KIMI, prefix_len=[1500, 70, 2049], parents=parents, seed=31)
+    a = datagen.make_case("a", **kw, paged=False)
+    b = datagen.make_case("b", **kw, paged=True)
+    for splits in (1, 0):
+        oa, la = _run(a, kdv.KDV_IMPL_TC, splits=splits)
+        ob, lb = _run(b, kdv.KDV_IMPL_TC, splits=splits)
+        np.testing.assert_array_equal(oa, ob)
+        np.testing.assert_array_equal(la, lb)
+    o_ref, lse_ref = oracle.verify_case(b)
+    assert_parity(ob, lb, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("L,T", [(0, 3), (5, 1), (127, 13), (300, 64)])
+def test_tc_paged_edges(L, T):
+    case = datagen.make_case("pe", **datagen.KIMI, prefix_len=[L],
+                             parents=[datagen.random_tree(T, np.random.default_rng(L))], seed=L + 5,
+                             paged=True)
+    o, lse = _run(case, kdv.KDV_IMPL_TC, splits=0)
+    o_ref, lse_ref = oracle.verify_case(case)
+    assert_parity(o, lse, o_ref, lse_ref)
+
+
+def test_tc_paged_bad_slot_reported():
+    case = datagen.make_case("bs", **datagen.KIMI, prefix_len=[200],
+                             parents=[datagen.chain_tree(4)], seed=9, paged=True)
+    case.page_table = case.page_table.copy()
+    case.page_table[17] = case.kv.shape[0] + 5          # outside the pool
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC, num_splits=1).run()
+    dc.results()
+    assert dc.error_flag() == kdv.KDV_DERR_BAD_SLOT
+
+
+def test_tc_auto_picks_tc_for_paged():
+    case = datagen.make_case("ap", **datagen.KIMI, prefix_len=[100],
+                             parents=[datagen.chain_tree(3)], seed=2, paged=True)
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_AUTO, num_splits=0)
+    plan = kdv.kdv_verify_attn_plan(dc.params)
+    dc_tc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC, num_splits=0)
+    assert plan == kdv.kdv_verify_attn_plan(dc_tc.params)
+    o, lse = dc.run().results()
+    o2, lse2 = dc_tc.run().results()
+    np.testing.assert_array_equal(o, o2)
+
+
+def test_tc_1sm_rejects_page_table():
+    case = datagen.make_case("r", **datagen.KIMI, prefix_len=[10], parents=[datagen.chain_tree(2)],
+                             seed=1, paged=True)
+    with pytest.raises(kdv.KdvError) as e:
+        kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_1SM).run()
+    assert e.value.status == kdv.KDV_ERR_UNSUPPORTED
