@@ -53,14 +53,52 @@ def workload_case(layer: int):
     return datagen.kimi_layer_case(L=L_PREFIX, T=T_TREE, seed=seed, tree_seed=1)
 
 
+SWEEP_L = (13, 1663, 3333, 5553)
+WORKLOADS = {
+    "kimi": "Kimi-shape layer, L=5553, T=13 random tree, NL layers per step",
+    "sweep": "context sweep, T=15 shared tree, L in {13, 1663, 3333, 5553}, NL layers per step",
+    "long": "L=200,000, T=16, KV ~ N(0,1), one layer per step",
+    "paged": "8 requests, L_b ~ U[1024, 32768], T_b ~ U[9, 16], page_size-1 pool through a "
+             "random-permutation page table, one batch per step",
+}
+
+
+def workload_cases(name: str, layers: int, rank: int = 0, world: int = 1, L: int = L_PREFIX):
+    """The list of verify problems one step runs (one kdv_verify_attn call each)."""
+    from speculative_tree_verify_mla_b200 import datagen
+    if name == "kimi":
+        return [workload_case(rank * 10_000 + l if world > 1 else l) for l in range(layers)]
+    if name == "sweep":
+        return [datagen.context_sweep_case(L, l + 100 * rank) for l in range(layers)]
+    if name == "long":
+        return [datagen.long_context_case()]
+    if name == "paged":
+        return [datagen.batched_paged_case(seed=4 + 1000 * rank)]
+    raise ValueError(name)
+
+
+def workload_name(name: str, L: int = L_PREFIX) -> str:
+    return {"kimi": f"kimi_layer_L{L_PREFIX}_T{T_TREE}", "sweep": f"context_sweep_L{L}_T15",
+            "long": "long_context_L200000_T16", "paged": "batched_paged_B8"}[name]
+
+
+def case_flops_bytes(case):
+    """Algorithmic work of one verify call: 2176 FLOPs per (row, visible key),
+    tree keys counted at their true visible count; 1152 B per KV row read once."""
+    flops, kv_bytes = 0.0, 0.0
+    for b in range(case.batch):
+        t0, t1 = int(case.tree_off[b]), int(case.tree_off[b + 1])
+        par, T, L = case.parent[t0:t1], t1 - t0, int(case.prefix_len[b])
+        depth = np.zeros(T, dtype=np.int64)      # |Anc*(t)| = depth(t) + 1
+        for t in range(1, T):
+            depth[t] = depth[par[t]] + 1 if par[t] >= 0 else 0
+        flops += case.H * (T * L + int((depth + 1).sum())) * FLOP_PER_ROW_KEY
+        kv_bytes += (L + T) * KV_ROW_BYTES
+    return float(flops), float(kv_bytes)
+
+
 def layer_flops_bytes(case):
-    T, H, L = int(case.tree_T[0]), case.H, int(case.prefix_len[0])
-    # |Anc*(t)| = depth(t) + 1, from parent[] (parents precede children)
-    depth = np.zeros(T, dtype=np.int64)
-    for t in range(1, T):
-        depth[t] = depth[case.parent[t]] + 1 if case.parent[t] >= 0 else 0
-    visible = H * (T * L + int((depth + 1).sum()))
-    return float(visible * FLOP_PER_ROW_KEY), float((L + T) * KV_ROW_BYTES)
+    return case_flops_bytes(case)
 
 
 def load_peaks():
@@ -174,7 +212,8 @@ def run_reference(args):
     import oracle
     oracle.build()
     cores = os.cpu_count()
-    case = workload_case(0)
+    L_main = args.sweep_L if args.workload == "sweep" else L_PREFIX
+    case = workload_cases(args.workload, 1, 0, 1, L_main)[0]
     rows_total = case.rows
     # size the per-step sample so the whole run stays within ~2 minutes
     dt1, *_ = time_oracle(case, 32)
@@ -193,11 +232,12 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": us_per_layer / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"kimi_layer_L{L_PREFIX}_T{T_TREE}", "H": 64, "d_latent": 512,
-                   "d_rope": 64, "prefix_len": L_PREFIX, "tree_nodes": T_TREE},
+        "config": {"workload": workload_name(args.workload, L_main), "H": 64, "d_latent": 512,
+                   "d_rope": 64, "prefix_len": [int(x) for x in case.prefix_len],
+                   "tree_nodes": [int(x) for x in case.tree_T]},
         "cpu_baseline": {"value": us_per_layer, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{n_rows} of {rows_total} query rows of layer 0 per step, "
-                                   "scaled to a full layer"},
+                         "sample": f"{n_rows} of {rows_total} query rows of the first call per "
+                                   "step, scaled to the whole call"},
         "e2e": {"value": us_per_layer, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -207,6 +247,100 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # GPU arm
 # --------------------------------------------------------------------------
+class Problems:
+    """The step's verify problems, resident on the device: one kdv_verify_attn
+    call per case (inputs, outputs, workspace), masks shared by cases whose
+    trees are identical, and a partials-out twin of every call for timing the
+    tensor-core kernel alone."""
+
+    def __init__(self, cases, impl_code, dev):
+        import torch
+        from speculative_tree_verify_mla_b200 import kdv
+        self.cases = cases
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        self.d_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.trees = {}          # tree bytes -> (parent, tree_off, batch, max_T, mask)
+        self.q, self.kv, self.o, self.lse, self.ws, self.params, self.tc_params = [], [], [], [], [], [], []
+        self.page_table, self.kv_off, self.tree_off, self.keep = [], [], [], []
+        self.splits, self.items, self.n_combine = [], [], 0
+        for c in cases:
+            key = c.parent.tobytes() + c.tree_off.tobytes()
+            if key not in self.trees:
+                sumT = int(c.tree_off[-1])
+                self.trees[key] = (i32(c.parent), i32(c.tree_off), c.batch, int(max(c.tree_T)),
+                                   torch.zeros(sumT, dtype=torch.int64, device=dev))
+            mask = self.trees[key][4]
+            q = torch.from_numpy(c.q).to(torch.bfloat16).to(dev)
+            kv = torch.from_numpy(c.kv).to(torch.bfloat16).to(dev)
+            pt = i32(c.page_table) if c.page_table is not None else None
+            kv_off, tree_off, plen = i32(c.kv_off), i32(c.tree_off), i32(c.prefix_len)
+            o = torch.empty(c.rows, 512, dtype=torch.float32, device=dev)
+            lse = torch.empty(c.rows, dtype=torch.float32, device=dev)
+            common = dict(batch=c.batch, num_heads=c.H, d_latent=512, d_rope=64, scale=c.scale,
+                          dtype=kdv.KDV_BF16, impl=impl_code, q=q, q_row_stride=576, kv=kv,
+                          num_slots=kv.shape[0], page_table=pt, kv_off=kv_off, tree_off=tree_off,
+                          prefix_len=plen, h_prefix_len=[int(x) for x in c.prefix_len],
+                          h_tree_T=[int(x) for x in c.tree_T], mask=mask, d_err=self.d_err)
+            p = kdv.make_params(**common, num_splits=0, return_partials=0, o=o, lse=lse,
+                                o_part=None, lse_part=None, workspace=None, workspace_bytes=0)
+            nbytes = kdv.kdv_verify_attn_workspace(p)
+            ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
+            p.workspace, p.workspace_bytes = ws.data_ptr(), nbytes
+            splits, items = kdv.kdv_verify_attn_plan(p)
+            if max(splits) > 1:
+                self.n_combine += 1
+            # partials-out twin (uniform S = the largest planned split count)
+            S = max(splits)
+            o_part = torch.empty(S, c.rows, 512, dtype=torch.float32, device=dev)
+            lse_part = torch.empty(S, c.rows, dtype=torch.float32, device=dev)
+            tp = kdv.make_params(**common, num_splits=S, return_partials=1, o=None, lse=None,
+                                 o_part=o_part, lse_part=lse_part, workspace=None,
+                                 workspace_bytes=0)
+            self.keep += [o_part, lse_part, plen]
+            self.q.append(q); self.kv.append(kv); self.o.append(o); self.lse.append(lse)
+            self.ws.append(ws); self.params.append(p); self.tc_params.append(tp)
+            self.page_table.append(pt); self.kv_off.append(kv_off); self.tree_off.append(tree_off)
+            self.splits.append(splits); self.items.append(items)
+
+    def step(self, s):
+        from speculative_tree_verify_mla_b200 import kdv
+        for parent, tree_off, B, max_T, mask in self.trees.values():
+            kdv.kdv_tree_mask_build(parent, tree_off, B, max_T, mask, None, self.d_err, s)
+        for p in self.params:
+            kdv.kdv_verify_attn(p, s)
+
+    def tc_only(self, s):
+        from speculative_tree_verify_mla_b200 import kdv
+        for p in self.tc_params:
+            kdv.kdv_verify_attn(p, s)
+
+    def launches_per_step(self):
+        return len(self.trees) + len(self.params) + self.n_combine
+
+
+def graph_of(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(stream)
+    return g
+
+
+def replay_us(g, stream, reps):
+    """Mean device time of one replay of graph g (CUDA events on `stream`)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
 def run_gpu(args):
     import torch
     from speculative_tree_verify_mla_b200 import kdv
@@ -221,74 +355,25 @@ def run_gpu(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     kdv.load()
-    NL = args.layers
     stream = torch.cuda.Stream(device=dev)
+    NL = args.layers if args.workload in ("kimi", "sweep") else 1
+    L_main = args.sweep_L if args.workload == "sweep" else L_PREFIX
 
     # ---- inputs (resident in HBM before timing) ----
-    cases = [workload_case(rank * 10_000 + l if world > 1 else l) for l in range(NL)]
-    c0 = cases[0]
-    T, H = int(c0.tree_T[0]), c0.H
-    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
-    parent = i32(c0.parent)
-    tree_off = i32(c0.tree_off)
-    kv_off = i32(c0.kv_off)
-    prefix_len = i32(c0.prefix_len)
-    mask = torch.zeros(T, dtype=torch.int64, device=dev)
-    d_err = torch.zeros(1, dtype=torch.int32, device=dev)
-    qs, kvs, outs, lses, wss, params, tc_params = [], [], [], [], [], [], []
-    common = dict(batch=1, num_heads=H, d_latent=512, d_rope=64, scale=c0.scale, dtype=kdv.KDV_BF16,
-                  q_row_stride=576, page_table=None, kv_off=kv_off, tree_off=tree_off,
-                  prefix_len=prefix_len, h_prefix_len=[L_PREFIX], h_tree_T=[T], mask=mask,
-                  d_err=d_err)
-    for c in cases:
-        q = torch.from_numpy(c.q).to(torch.bfloat16).to(dev)
-        kv = torch.from_numpy(c.kv).to(torch.bfloat16).to(dev)
-        o = torch.empty(c.rows, 512, dtype=torch.float32, device=dev)
-        lse = torch.empty(c.rows, dtype=torch.float32, device=dev)
-        p = kdv.make_params(**common, impl=args.impl_code, q=q, kv=kv, num_slots=kv.shape[0],
-                            num_splits=0, return_partials=0, o=o, lse=lse, o_part=None,
-                            lse_part=None, workspace=None, workspace_bytes=0)
-        nbytes = kdv.kdv_verify_attn_workspace(p)
-        ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
-        p.workspace, p.workspace_bytes = ws.data_ptr(), nbytes
-        qs.append(q); kvs.append(kv); outs.append(o); lses.append(lse); wss.append(ws); params.append(p)
-    splits, items = kdv.kdv_verify_attn_plan(params[0])
-    S = splits[0]
-    o_part = torch.empty(S, c0.rows, 512, dtype=torch.float32, device=dev)
-    lse_part = torch.empty(S, c0.rows, dtype=torch.float32, device=dev)
-    for l, c in enumerate(cases):
-        tc_params.append(kdv.make_params(**common, impl=args.impl_code, q=qs[l], kv=kvs[l],
-                                         num_slots=kvs[l].shape[0], num_splits=S, return_partials=1,
-                                         o=None, lse=None, o_part=o_part, lse_part=lse_part,
-                                         workspace=None, workspace_bytes=0))
-
-    def step(s):
-        kdv.kdv_tree_mask_build(parent, tree_off, 1, T, mask, None, d_err, s)
-        for p in params:
-            kdv.kdv_verify_attn(p, s)
-
-    def tc_only(s):
-        for p in tc_params:
-            kdv.kdv_verify_attn(p, s)
-
-    # eager warm-up (sets kernel attributes), then capture graphs
-    with torch.cuda.stream(stream):
-        step(stream)
-        tc_only(stream)
+    prob = Problems(workload_cases(args.workload, NL, rank, world, L_main), args.impl_code, dev)
+    c0 = prob.cases[0]
+    with torch.cuda.stream(stream):        # eager warm-up sets kernel attributes
+        prob.step(stream)
+        prob.tc_only(stream)
     stream.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=stream):
-        step(stream)
-    g_tc = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_tc, stream=stream):
-        tc_only(stream)
+    g_step = graph_of(prob.step, stream)
+    g_tc = graph_of(prob.tc_only, stream)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(dev.index if world == 1 else local)
     sampler.start()
     time.sleep(0.3)
-    # graph replays and the timing events all go on `stream`
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream):        # graph replays and events all go on `stream`
         for _ in range(args.warmup):
             g_step.replay()
     torch.cuda.synchronize()
@@ -311,50 +396,54 @@ def run_gpu(args):
     ms_per_step = ms_total / args.steps
 
     # dominant kernel alone (same grid, partials out): per-launch duration
-    reps = max(3, min(50, args.steps // 4))
-    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            g_tc.replay()
-        e2.record(stream)
-        for _ in range(reps):
-            g_tc.replay()
-        e3.record(stream)
-    torch.cuda.synchronize()
-    tc_us = e2.elapsed_time(e3) * 1e3 / (reps * NL)
+    tc_us = replay_us(g_tc, stream, max(3, min(50, args.steps // 4))) / len(prob.params)
     clocks = sampler.stop()
-    assert int(d_err.item()) == 0, f"device error flag {int(d_err.item())}"
+    assert int(prob.d_err.item()) == 0, f"device error flag {int(prob.d_err.item())}"
 
-    # eager (stream-ordered, no graph) per-layer time, for reference
+    # eager (stream-ordered, no graph) per-call time, for reference
     with torch.cuda.stream(stream):
         e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e4.record(stream)
         for _ in range(3):
-            step(stream)
+            prob.step(stream)
         e5.record(stream)
     torch.cuda.synchronize()
-    eager_us = e4.elapsed_time(e5) * 1e3 / (3 * NL)
+    eager_us = e4.elapsed_time(e5) * 1e3 / (3 * len(prob.params))
 
-    # ---- end to end through the C ABI with host buffers ----
+    # ---- end to end through the C ABI with host buffers: the step's tree
+    # (parent[]), every query row and the tree nodes' own KV rows go up, o and
+    # lse come back ----
     pin = lambda t: t.cpu().pin_memory()
-    h_parent = pin(parent)
-    h_q = [pin(q) for q in qs]
-    h_tree_kv = [pin(kv[L_PREFIX:L_PREFIX + T]) for kv in kvs]
-    h_o = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h_l = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in lses]
-    h2d = h_parent.numel() * 4 + sum(x.numel() * 2 for x in h_q) + sum(x.numel() * 2 for x in h_tree_kv)
+    h_parent = [pin(tr[0]) for tr in prob.trees.values()]
+    h_q = [pin(q) for q in prob.q]
+    up_rows = []                 # (device row view, pinned host copy) of the tree-node KV rows
+    for c, kv, pt in zip(prob.cases, prob.kv, prob.page_table):
+        for b in range(c.batch):
+            L, T, k0 = int(c.prefix_len[b]), int(c.tree_T[b]), int(c.kv_off[b])
+            if c.page_table is None:
+                up_rows.append((kv[k0 + L:k0 + L + T], pin(kv[k0 + L:k0 + L + T])))
+            else:
+                for u in range(T):
+                    slot = int(c.page_table[k0 + L + u])
+                    up_rows.append((kv[slot:slot + 1], pin(kv[slot:slot + 1])))
+    h_o = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in prob.o]
+    h_l = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in prob.lse]
+    h2d = (sum(x.numel() * 4 for x in h_parent) + sum(x.numel() * 2 for x in h_q)
+           + sum(h.numel() * 2 for _, h in up_rows))
     d2h = sum(x.numel() * 4 for x in h_o) + sum(x.numel() * 4 for x in h_l)
 
     def e2e_step():
         with torch.cuda.stream(stream):
-            parent.copy_(h_parent, non_blocking=True)
-            for l in range(NL):
-                qs[l].copy_(h_q[l], non_blocking=True)
-                kvs[l][L_PREFIX:L_PREFIX + T].copy_(h_tree_kv[l], non_blocking=True)
-            step(stream)
-            for l in range(NL):
-                h_o[l].copy_(outs[l], non_blocking=True)
-                h_l[l].copy_(lses[l], non_blocking=True)
+            for tr, hp in zip(prob.trees.values(), h_parent):
+                tr[0].copy_(hp, non_blocking=True)
+            for q, hq in zip(prob.q, h_q):
+                q.copy_(hq, non_blocking=True)
+            for d, h in up_rows:
+                d.copy_(h, non_blocking=True)
+            prob.step(stream)
+            for o, ho, l, hl in zip(prob.o, h_o, prob.lse, h_l):
+                ho.copy_(o, non_blocking=True)
+                hl.copy_(l, non_blocking=True)
         stream.synchronize()
 
     e2e_steps = max(2, min(10, args.steps))
@@ -374,36 +463,47 @@ def run_gpu(args):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
-    flops, kv_bytes = layer_flops_bytes(c0)
+    flops, kv_bytes = case_flops_bytes(c0)
     peaks = load_peaks()
-    us_per_layer = ms_per_step * 1e3 / (NL * world)
+    n_calls = len(prob.params)
+    us_per_call = ms_per_step * 1e3 / (n_calls * world)
     tc_tflops = flops / (tc_us * 1e-6) / 1e12
     kname, ksrc = TC_KERNEL.get(args.impl_code, TC_KERNEL[2])
-    traffic = load_traffic(kname, ksrc)
+    traffic = load_traffic(kname, ksrc) if args.workload == "kimi" else None
     roof_us = max(flops / (peaks["bf16_tflops"] * 1e12), kv_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+    workload = workload_name(args.workload, L_main)
+    if args.workload == "kimi":
+        cfg = {"workload": workload, "H": c0.H, "d_latent": 512, "d_rope": 64, "d_nope": 128,
+               "d_v": 128, "prefix_len": L_PREFIX, "tree_nodes": int(c0.tree_T[0]),
+               "layers_per_step": NL}
+    else:
+        cfg = {"workload": workload, "description": WORKLOADS[args.workload], "H": c0.H,
+               "d_latent": 512, "d_rope": 64, "prefix_len": [int(x) for x in c0.prefix_len],
+               "tree_nodes": [int(x) for x in c0.tree_T], "calls_per_step": n_calls}
+    step_bytes = n_calls * kv_bytes
+    cfg.update({"splits": prob.splits[0], "grid_items": prob.items[0],
+                "l2": (f"{n_calls} distinct KV caches ({step_bytes / 1e6:.0f} MB) per step > 126 MB L2"
+                       if step_bytes > 126e6 else
+                       f"KV {step_bytes / 1e6:.0f} MB per step fits L2: warm-L2 number"),
+                "timing": "CUDA graph replay of the step, CUDA events on the launch stream",
+                "parallelism": f"replica{world}" if world > 1 else "single"})
     result = {
-        "metric": METRIC, "value": us_per_layer, "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": us_per_call, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": f"kimi_layer_L{L_PREFIX}_T{T_TREE}", "H": H, "d_latent": 512,
-                   "d_rope": 64, "d_nope": 128, "d_v": 128, "prefix_len": L_PREFIX,
-                   "tree_nodes": T, "layers_per_step": NL, "splits": S, "grid_items": items,
-                   "l2": f"{NL} distinct KV caches ({NL * kv_bytes / 1e6:.0f} MB) per step > 126 MB L2",
-                   "timing": "CUDA graph replay of the step, CUDA events on the launch stream",
-                   "parallelism": f"replica{world}" if world > 1 else "single"},
-        "tflops_per_layer": flops / (us_per_layer * 1e-6) / 1e12,
+        "data": "synthetic", "config": cfg,
+        "tflops_per_layer": flops / (us_per_call * 1e-6) / 1e12,
         "roofline_us_per_layer": roof_us,
-        "frac_of_roofline": roof_us / us_per_layer,
+        "frac_of_roofline": roof_us / us_per_call,
         "eager_us_per_layer": eager_us,
         "roofline": {"bound": "tensor", "kernel": kname, "achieved": tc_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tc_tflops / peaks["bf16_tflops"], "traffic": traffic,
                      "us_per_launch": tc_us, "flops_per_launch": flops,
                      "kv_bytes_per_launch": kv_bytes, "peak_source": peaks["source"] + " burst bf16"},
-        "e2e": {"value": e2e_ms * 1e3 / NL, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        "e2e": {"value": e2e_ms * 1e3 / n_calls, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": args.steps * (1 + 2 * NL) if S > 1 else args.steps * (1 + NL),
+        "gpu_launches": args.steps * prob.launches_per_step(),
         "clocks": clocks,
     }
 
@@ -411,17 +511,17 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        dt1, *_ = time_oracle(c0, 64)
-        n_rows = int(min(c0.rows, max(64, 15.0 / max(dt1 / 64, 1e-6))))
+        dt1, *_ = time_oracle(c0, 16)
+        n_rows = int(min(c0.rows, max(16, 15.0 / max(dt1 / 16, 1e-6))))
         dt, rows, o_ref, l_ref = time_oracle(c0, n_rows)
         cpu_us = dt / n_rows * c0.rows * 1e6
         result["cpu_baseline"] = {"value": cpu_us, "unit": UNIT, "cores": os.cpu_count(),
                                   "kind": "oracle",
-                                  "sample": f"{n_rows} of {c0.rows} query rows of layer 0 "
-                                            "(fp64, all keys), scaled to a full layer"}
+                                  "sample": f"{n_rows} of {c0.rows} query rows of the first call "
+                                            "(fp64, all keys), scaled to the whole call"}
         from tests.parity import parity_stats
-        got_o = outs[0].cpu().numpy()[rows]
-        got_l = lses[0].cpu().numpy()[rows]
+        got_o = prob.o[0].cpu().numpy()[rows]
+        got_l = prob.lse[0].cpu().numpy()[rows]
         st = parity_stats(got_o, got_l, o_ref, l_ref)
         result["parity_layer0"] = {k: float(f"{v:.3g}") for k, v in st.items()}
     if rank == 0:
@@ -442,6 +542,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", choices=["tc2", "tc1"], default="tc2",
                     help="tensor-core kernel: 2-SM MMAs (default) or 1-SM MMAs")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kimi",
+                    help="kimi (default, the headline): " + WORKLOADS["kimi"] + "; sweep: "
+                         + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
+                         + "; paged: " + WORKLOADS["paged"])
+    ap.add_argument("--sweep-L", type=int, choices=SWEEP_L, default=5553)
     args = ap.parse_args()
     args.impl_code = 2 if args.kernel == "tc2" else 3
     args.warmup = max(3, args.warmup)

@@ -97,7 +97,6 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   plan->H = H;
   plan->rows_per_tile = rows_per_tile;
   int64_t tree_acc = 0;
-  double work = 0.0;
   for (int b = 0; b < B; ++b) {
     plan->L[b] = p->h_prefix_len[b];
     plan->T[b] = p->h_tree_T[b];
@@ -107,7 +106,6 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
     const int64_t tiles = (rows_b + rows_per_tile - 1) / rows_per_tile;
     if (tiles > INT_MAX / 2 || rows_b > INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
     plan->tiles[b] = (int32_t)tiles;
-    work += (double)tiles * ((double)p->h_prefix_len[b] + p->h_tree_T[b]);
   }
   if (tree_acc * (int64_t)H > INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
   plan->total_rows = (int32_t)(tree_acc * H);
@@ -126,15 +124,55 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
     target_items = n > 0 ? n : sms / 2;
   }
   const int min_keys = is_tc(impl) ? 2 * TC_KEYS : 128;
+  // Automatic splits: choose the chunk X (a multiple of SPLIT_ALIGN keys, at
+  // least min_keys) that minimises a simple cost model of the kernel, in
+  // units of keys processed by one work item:
+  //   items(X) = sum_b tiles_b * ceil(n_b / X)
+  //   one wave  (items <= clusters): the longest item, X + C
+  //   more waves: (sum_b tiles_b * n_b + items * C) / clusters + (X + C) / 2
+  // C = ITEM_OVERHEAD_KEYS is the fixed cost of an item (query load, pipeline
+  // fill, epilogue and the partials it writes) measured on B200 as ~20 us
+  // against ~7 us per 256 keys of steady-state work, i.e. ~740 keys.
+  constexpr double ITEM_OVERHEAD_KEYS = 768.0;
+  int64_t max_n = 1;
+  double work_keys = 0.0;
+  for (int b = 0; b < B; ++b) {
+    max_n = std::max<int64_t>(max_n, (int64_t)plan->L[b] + plan->T[b]);
+    work_keys += (double)plan->tiles[b] * ((double)plan->L[b] + plan->T[b]);
+  }
+  auto items_for = [&](int64_t X) {
+    double n = 0.0;
+    for (int b = 0; b < B; ++b)
+      n += (double)plan->tiles[b] * (double)(((int64_t)plan->L[b] + plan->T[b] + X - 1) / X);
+    return n;
+  };
+  auto cost = [&](int64_t X) {
+    const double n = items_for(X), C = ITEM_OVERHEAD_KEYS;
+    if (n <= target_items) return (double)X + C;
+    return (work_keys + n * C) / target_items + 0.5 * ((double)X + C);
+  };
+  const int64_t align = SPLIT_ALIGN;
+  const int64_t x_lo = std::max<int64_t>(min_keys, align);
+  const int64_t x_hi = std::max<int64_t>(x_lo, ((max_n + align - 1) / align) * align);
+  int64_t best_x = x_hi;
+  double best_cost = cost(x_hi);
+  for (double xf = (double)x_lo; xf < (double)x_hi; xf *= 1.05) {     // ~100 candidates
+    const int64_t X = std::max(x_lo, ((int64_t)xf / align) * align);
+    const double cx = cost(X);
+    if (cx < best_cost) {
+      best_cost = cx;
+      best_x = X;
+    }
+  }
+  const int64_t hi = best_x;
+  const int64_t X = hi;
   for (int b = 0; b < B; ++b) {
     const int64_t n_b = (int64_t)plan->L[b] + plan->T[b];
     int64_t S;
     if (p->num_splits >= 1) {
       S = p->num_splits;
     } else {
-      const double per_item = work / target_items;          // keys x tiles per item
-      S = (int64_t)std::floor((double)n_b * plan->tiles[b] / std::max(per_item, 1.0) / plan->tiles[b]);
-      S = std::max<int64_t>(1, std::min<int64_t>(S, (n_b + min_keys - 1) / min_keys));
+      S = std::max<int64_t>(1, (n_b + X - 1) / X);
     }
     if (S > 4096) return KDV_ERR_UNSUPPORTED;
     const int64_t chunk = SPLIT_ALIGN * ((n_b + SPLIT_ALIGN * S - 1) / (SPLIT_ALIGN * S));

@@ -95,8 +95,9 @@ constexpr int OFF_XCHG = OFF_QROPE + QBLOCK_BYTES;           // float [2][2][128
 constexpr int XCHG_BYTES = 5 * ROWS * 4;
 constexpr int OFF_P = V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
+constexpr int OFF_VSLOT = OFF_STATS + STATS_BYTES;            // int32 [256] (O side, paged KV)
 constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
-static_assert(OFF_STATS + STATS_BYTES <= OFF_MISC, "O-side buffers overlap misc");
+static_assert(OFF_VSLOT + STILE * 4 <= OFF_MISC, "O-side buffers overlap misc");
 constexpr int OFF_BAR = OFF_MISC;
 constexpr int NUM_BARS = 48;
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
@@ -290,7 +291,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // barriers). Paged KV: the whole warp gathers, 4 rows per lane.
       const int n_stg = n_stiles * STAGES_PER_TILE;
       int issued = 0;
-      int32_t slot[4] = {0, 0, 0, 0};
+      // paged KV: lane l gathers keys 4l..4l+3 of this CTA's 128; their slots
+      // are read one tile ahead so the page-table latency stays off the path
+      int32_t slot[4] = {0, 0, 0, 0}, nslot[4] = {0, 0, 0, 0};
+      if (PAGED && n_stiles > 0) {
+        const int j0 = stile_key(0) + (int)half * HKEYS + 4 * lane;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
+      }
       if (n_stiles > 0 && lane == 0) {
         const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
         mbar_arrive_expect_tx(c.bar(B_QLAT_FULL), QLAT_BLOCKS * QBLOCK_BYTES);
@@ -310,9 +318,13 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const uint32_t dst = base + OFF_RING + st * KV_STAGE_BYTES;
         if (PAGED) {
           if (g % STAGES_PER_TILE == 0) {
-            const int j0 = stile_key(tile) + (int)half * HKEYS + 4 * lane;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) slot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
+            for (int q = 0; q < 4; ++q) slot[q] = nslot[q];
+            if (tile + 1 < n_stiles) {
+              const int j0 = stile_key(tile + 1) + (int)half * HKEYS + 4 * lane;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
+            }
           }
           for (int e = 0; e < STAGE_BLOCKS; ++e)
             tma_gather4_pair(dst + e * KBLOCK_BYTES + lane * 512, &tmap_kv, fb, (blk0 + e) * 64, slot[0], slot[1],
@@ -512,6 +524,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // Paged KV: lanes 0-7 gather 4 rows each.
       int issued = 0;
       const int n_sub = (KEYS / VKEYS) * n_ptiles;
+      // paged KV: the 256 slots of an S tile sit in a shared table (lane l
+      // reads keys 8l..8l+7 of the next tile one tile ahead, in registers)
+      int32_t* vslot = reinterpret_cast<int32_t*>(smem + OFF_VSLOT);
+      int32_t nv[8];
+      if (PAGED && n_stiles > 0) {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) nv[m] = paged_slot(a, kv_base, stile_key(0) + 8 * lane + m, k_hi);
+      }
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
         const uint32_t eparity = ((u / V_STAGES) & 1) ^ 1;
@@ -522,10 +542,21 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const uint32_t dst = base + OFF_RING + st * V_STAGE_BYTES;
         const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
         if (PAGED) {
+          const int vt = u / (STILE / VKEYS);
+          if (u % (STILE / VKEYS) == 0) {          // entering S tile vt: publish its slots
+#pragma unroll
+            for (int m = 0; m < 8; ++m) vslot[8 * lane + m] = nv[m];
+            if (vt + 1 < n_stiles) {
+#pragma unroll
+              for (int m = 0; m < 8; ++m) nv[m] = paged_slot(a, kv_base, stile_key(vt + 1) + 8 * lane + m, k_hi);
+            }
+            __syncwarp();
+          }
           if (lane < VKEYS / 4) {
+            const int k = key0 - stile_key(vt) + 4 * lane;
             int32_t slot[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) slot[q] = paged_slot(a, kv_base, key0 + 4 * lane + q, k_hi);
+            for (int q = 0; q < 4; ++q) slot[q] = vslot[k + q];
             for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
               const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
               tma_gather4_pair(dst + lb * VBLOCK_BYTES + lane * 512, &tmap_v, fb, gb * 64, slot[0], slot[1], slot[2],
