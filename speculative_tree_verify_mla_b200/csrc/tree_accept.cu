@@ -9,8 +9,9 @@
 //       of one row to one 64-bit key (orderable value << 32 | ~index), so a
 //       plain unsigned max picks the largest value and, among equal values,
 //       the lowest index. HBM-bound: it streams the logits once.
-//   accept_tree_kernel     one CTA of 64 threads per request (thread = node):
-//       finishes the argmax over the chunk keys, decides for every node
+//   accept_tree_kernel     one CTA of 256 threads per request: the warps
+//       finish the argmax over the chunk keys (one node per warp at a time),
+//       then thread t <-> node t (warps 0-1) decides for every node
 //       whether its root path is accepted (each node walks its own ancestors,
 //       so no node waits on another), takes the deepest accepted node (lowest
 //       index on ties), writes the path, the bonus token and optionally
@@ -24,7 +25,8 @@ namespace {
 
 constexpr int ARGMAX_THREADS = 256;
 constexpr int CHUNK = 8192;          // logits per argmax CTA
-constexpr int ACCEPT_THREADS = 64;   // = KDV_MAX_TREE
+constexpr int ACCEPT_THREADS = 256;  // 8 warps reduce the chunk keys; warps 0-1 hold the nodes
+constexpr int MAX_NODES = 64;        // = KDV_MAX_TREE
 
 __device__ __forceinline__ void record_err(int32_t* d_err, int32_t code) {
   if (d_err != nullptr) atomicCAS(d_err, 0, code);
@@ -50,7 +52,32 @@ argmax_partial_kernel(const void* __restrict__ logits, int64_t ld, int32_t vocab
   const int64_t c0 = (int64_t)chunk * CHUNK;
   const int64_t c1 = c0 + CHUNK < vocab ? c0 + CHUNK : vocab;
   unsigned long long best = 0ull;
-  if (BF16) {
+  const bool full = vec && c1 - c0 == CHUNK;
+  if (full) {
+    // a whole chunk: every thread issues all its 16-byte loads before using
+    // any, so the CTA costs one memory round trip
+    constexpr int LOADS = CHUNK * (BF16 ? 2 : 4) / 16 / ARGMAX_THREADS;
+    constexpr int PER = BF16 ? 8 : 4;                 // logits per load
+    const uint4* x4 = reinterpret_cast<const uint4*>(static_cast<const char*>(logits) +
+                                                     ((int64_t)row * ld + c0) * (BF16 ? 2 : 4));
+    uint4 u[LOADS];
+#pragma unroll
+    for (int k = 0; k < LOADS; ++k) u[k] = __ldg(x4 + k * ARGMAX_THREADS + threadIdx.x);
+#pragma unroll
+    for (int k = 0; k < LOADS; ++k) {
+      const uint32_t idx0 = (uint32_t)(c0 + (int64_t)(k * ARGMAX_THREADS + threadIdx.x) * PER);
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (BF16) {
+          best = umax64(best, logit_key(w[q] << 16, idx0 + 2 * q));
+          best = umax64(best, logit_key(w[q] & 0xffff0000u, idx0 + 2 * q + 1));
+        } else {
+          best = umax64(best, logit_key(w[q], idx0 + q));
+        }
+      }
+    }
+  } else if (BF16) {
     const uint16_t* x = static_cast<const uint16_t*>(logits) + (int64_t)row * ld;
     if (vec) {
       // 8 logits per 16-byte load; the row start is 16-byte aligned and CHUNK
@@ -121,9 +148,10 @@ struct AcceptArgs {
 };
 
 __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const AcceptArgs a) {
-  __shared__ int32_t s_parent[ACCEPT_THREADS], s_token[ACCEPT_THREADS], s_target[ACCEPT_THREADS];
-  __shared__ int32_t s_path[ACCEPT_THREADS];
+  __shared__ int32_t s_parent[MAX_NODES], s_token[MAX_NODES], s_target[MAX_NODES];
+  __shared__ int32_t s_path[MAX_NODES];
   __shared__ unsigned long long s_key[ACCEPT_THREADS / 32];
+  __shared__ int s_off_count;
   const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int t0 = a.tree_off[b];
   const int T = a.tree_off[b + 1] - t0;
@@ -138,27 +166,30 @@ __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const Accep
     if (t < a.max_T) path_out[t] = -1;
     return;
   }
-  // ---- per-node target and inputs
+  // ---- target of every node: warp w reduces the chunk keys of nodes w, w+8, ...
+  if (a.part != nullptr) {
+    for (int n = warp; n < T; n += ACCEPT_THREADS / 32) {
+      const unsigned long long* kp = a.part + (int64_t)(t0 + n) * a.chunks;
+      unsigned long long key = 0ull;
+      for (int c = lane; c < a.chunks; c += 32) key = umax64(key, kp[c]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) key = umax64(key, __shfl_xor_sync(0xffffffffu, key, o));
+      if (lane == 0) s_target[n] = key == 0ull ? 0 : (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffull));
+    }
+  } else if (t < T) {
+    const int32_t target = a.target_in[t0 + t];
+    if (target < 0 || target >= a.vocab) record_err(a.d_err, KDV_DERR_BAD_TOKEN);
+    s_target[t] = target;
+  }
+  // ---- per-node inputs (thread t <-> node t)
   bool bad_parent = false;
   if (t < T) {
-    const int row = t0 + t;
-    int32_t target;
-    if (a.part != nullptr) {
-      unsigned long long key = 0ull;
-      for (int c = 0; c < a.chunks; ++c) key = umax64(key, a.part[(int64_t)row * a.chunks + c]);
-      target = key == 0ull ? 0 : (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffull));
-    } else {
-      target = a.target_in[row];
-      if (target < 0 || target >= a.vocab) record_err(a.d_err, KDV_DERR_BAD_TOKEN);
-    }
-    const int32_t p = a.parent[row];
-    const int32_t tok = a.token[row];
+    const int32_t p = a.parent[t0 + t];
+    const int32_t tok = a.token[t0 + t];
     bad_parent = !(p == -1 || (p >= 0 && p < t));
     if (p != -1 && (tok < 0 || tok >= a.vocab)) record_err(a.d_err, KDV_DERR_BAD_TOKEN);
     s_parent[t] = p;
     s_token[t] = tok;
-    s_target[t] = target;
-    if (a.target_out) a.target_out[row] = target;
   }
   if (__syncthreads_or(bad_parent)) {
     if (t == 0) {
@@ -167,9 +198,11 @@ __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const Accep
       if (a.bonus) a.bonus[b] = -1;
       if (a.prefix_len_out) a.prefix_len_out[b] = a.prefix_len[b];
     }
+    if (t < T && a.target_out) a.target_out[t0 + t] = s_target[t];
     if (t < a.max_T) path_out[t] = -1;
     return;
   }
+  if (t < T && a.target_out) a.target_out[t0 + t] = s_target[t];
   // ---- accepted iff every edge on the root path matches; key = (depth+1, -t)
   unsigned long long key = 0ull;
   int depth = 0;
@@ -185,7 +218,9 @@ __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const Accep
   for (int o = 16; o > 0; o >>= 1) key = umax64(key, __shfl_xor_sync(0xffffffffu, key, o));
   if (lane == 0) s_key[warp] = key;
   __syncthreads();
-  const unsigned long long best = umax64(s_key[0], s_key[1]);
+  unsigned long long best = 0ull;
+#pragma unroll
+  for (int w = 0; w < ACCEPT_THREADS / 32; ++w) best = umax64(best, s_key[w]);
   const int end = 255 - (int)(best & 255ull);
   const int len = (int)(best >> 8);
   if (t == 0) {
@@ -207,7 +242,6 @@ __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const Accep
     const bool on_path = t < T && depth < len && s_path[depth] == t;
     const bool off_path = t < T && !on_path;
     const unsigned ballot = __ballot_sync(0xffffffffu, off_path);
-    __shared__ int s_off_count;
     if (t == 31) s_off_count = __popc(ballot);
     int32_t old = 0;
     if (t < T) old = a.page_table[base + t];

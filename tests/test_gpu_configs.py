@@ -1,0 +1,79 @@
+"""GPU parity at the full sizes of every workload, in the launch configuration
+the benchmark times (kdv_verify_attn, AUTO kernel, automatic splits).
+
+The oracle evaluates sampled query rows where all rows would take too long;
+rows are spread over every request, head and tree node. Tolerances are the
+stated bars (tests/parity.py).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from speculative_tree_verify_mla_b200 import datagen, kdv
+from tests.parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_rows(case, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(case.rows, size=min(n, case.rows), replace=False).tolist())
+    for b in range(case.batch):            # first and last row of every request
+        r = case.request_rows(b)
+        rows |= {r.start, r.stop - 1}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def _check(case, rows=None, **kw):
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_AUTO, num_splits=0).run()
+    o, lse = dc.results()
+    assert dc.error_flag() == 0
+    if rows is None:
+        o_ref, lse_ref = oracle.verify_case(case)
+        assert_parity(o, lse, o_ref, lse_ref, **kw)
+    else:
+        o_ref, lse_ref = oracle.verify_case(case, rows=rows)
+        assert_parity(o[rows], lse[rows], o_ref, lse_ref, **kw)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    return dc
+
+
+def test_config1_kimi_layer_all_rows():
+    """Kimi shape, L=5553, T=13: every one of the 832 rows."""
+    _check(datagen.kimi_layer_case(L=5553, T=13, seed=1))
+
+
+@pytest.mark.parametrize("L", datagen.CONTEXT_SWEEP)
+def test_config2_context_sweep(L):
+    """T=15 shared tree; layers 0, 30 and 60 of the 61."""
+    for layer in (0, 30, 60):
+        case = datagen.context_sweep_case(L, layer)
+        _check(case, rows=None if L <= 1663 else _sample_rows(case, 192, layer + L))
+
+
+def test_config3_long_context_200k():
+    """L=200,000, T=16, KV ~ N(0,1): split-L across SMs and the LSE merge."""
+    case = datagen.long_context_case()
+    dc = _check(case, rows=_sample_rows(case, 48, 3))
+    splits, _ = kdv.kdv_verify_attn_plan(dc.params)
+    assert splits[0] > 1                    # the split path is what ran
+
+
+def test_config4_batched_paged():
+    """8 requests, L_b ~ U[1024, 32768], T_b ~ U[9, 16], permuted pool."""
+    case = datagen.batched_paged_case()
+    assert case.page_table is not None
+    _check(case, rows=_sample_rows(case, 96, 4))
+
+
+def test_config4_matches_contiguous_bit_for_bit():
+    """The paged batch equals the same batch with a contiguous pool exactly."""
+    paged = datagen.batched_paged_case()
+    plen = [int(x) for x in paged.prefix_len]
+    parents = [paged.parent[paged.tree_off[b]:paged.tree_off[b + 1]] for b in range(paged.batch)]
+    flat = datagen.make_case("flat", **datagen.KIMI, prefix_len=plen, parents=parents, dtype="bf16",
+                             seed=paged.seed, paged=False)
+    a = kdv.DeviceCase(paged, num_splits=0).run().results()
+    b = kdv.DeviceCase(flat, num_splits=0).run().results()
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
