@@ -275,6 +275,28 @@ KDV_API kdv_status kdv_tree_accept_workspace(const kdv_accept_params* p, size_t*
  */
 KDV_API kdv_status kdv_tree_accept(const kdv_accept_params* p, void* stream);
 
+/*
+ * The two per-head projections around absorbed-form attention (the latent
+ * projection that page "The Architecture of Diagnosis", section "Phase 1:
+ * Custom CUDA Kernels", item 2 says the verify kernel absorbs):
+ *   kdv_absorb_q:   q_lat[row] = W_UK[h] q_nope[row]     (W_UK [H][D_c][D_n])
+ *   kdv_unabsorb_o: out[row]   = W_UV[h]^T o_lat[row]    (W_UV [H][D_c][D_v])
+ * Rows are node-major, row = t*H + h (rows must be a multiple of H). Weights
+ * and q_nope are KDV_BF16 or KDV_F32; o_lat is fp32 (kdv_verify_attn's
+ * output); out_dtype selects the output element type (KDV_BF16 rounds to
+ * nearest even). Strides are in elements: q_lat may be written straight into
+ * the first D_c columns of kdv_verify_attn's q rows (q_lat_stride = D_c +
+ * D_r). Accumulation is fp32. Limits: D_n <= 512, D_c <= 4096 (absorb);
+ * D_c <= 512, D_v <= 4096 (unabsorb); otherwise KDV_ERR_UNSUPPORTED.
+ */
+KDV_API kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope,
+                                const void* q_nope, int64_t q_nope_stride, int32_t q_dtype, const void* w_uk,
+                                int32_t w_dtype, void* q_lat, int64_t q_lat_stride, int32_t out_dtype,
+                                void* stream);
+KDV_API kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v,
+                                  const float* o_lat, int64_t o_lat_stride, const void* w_uv, int32_t w_dtype,
+                                  void* out, int64_t out_stride, int32_t out_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,7 +43,7 @@ KDV_MAX_BATCH = 128
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
             "kdv_verify_attn_noalloc", "kdv_combine", "kdv_tree_accept_workspace",
-            "kdv_tree_accept")
+            "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -125,6 +125,13 @@ def load() -> ctypes.CDLL:
         lib.kdv_tree_accept_workspace.restype = c.c_int
         lib.kdv_tree_accept.argtypes = [c.POINTER(AcceptParams), c.c_void_p]
         lib.kdv_tree_accept.restype = c.c_int
+        lib.kdv_absorb_q.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int32, c.c_void_p, c.c_int64,
+                                     c.c_int32, c.c_void_p, c.c_int32, c.c_void_p, c.c_int64, c.c_int32,
+                                     c.c_void_p]
+        lib.kdv_absorb_q.restype = c.c_int
+        lib.kdv_unabsorb_o.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int32, c.c_void_p, c.c_int64,
+                                       c.c_void_p, c.c_int32, c.c_void_p, c.c_int64, c.c_int32, c.c_void_p]
+        lib.kdv_unabsorb_o.restype = c.c_int
         _lib = lib
     return _lib
 
@@ -210,6 +217,34 @@ def kdv_verify_attn_noalloc(params: VerifyParams, stream=None) -> None:
     """kdv_verify_attn with the library's built-in scratch instead of params.workspace."""
     _check(load().kdv_verify_attn_noalloc(ctypes.byref(params), _stream(stream)),
            "kdv_verify_attn_noalloc")
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDV_BF16
+    if t.dtype == torch.float32:
+        return KDV_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def kdv_absorb_q(num_heads: int, q_nope: torch.Tensor, w_uk: torch.Tensor, q_lat: torch.Tensor,
+                 stream=None) -> None:
+    """q_lat[row, :D_c] = W_UK[row % H] q_nope[row] (2-D row-strided tensors)."""
+    rows, d_nope = q_nope.shape
+    d_latent = w_uk.shape[1]
+    _check(load().kdv_absorb_q(int(rows), int(num_heads), int(d_latent), int(d_nope), _ptr(q_nope),
+                               int(q_nope.stride(0)), _dt(q_nope), _ptr(w_uk), _dt(w_uk), _ptr(q_lat),
+                               int(q_lat.stride(0)), _dt(q_lat), _stream(stream)), "kdv_absorb_q")
+
+
+def kdv_unabsorb_o(num_heads: int, o_lat: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor,
+                   stream=None) -> None:
+    """out[row] = W_UV[row % H]^T o_lat[row] (o_lat fp32)."""
+    rows, d_latent = o_lat.shape
+    d_v = w_uv.shape[2]
+    _check(load().kdv_unabsorb_o(int(rows), int(num_heads), int(d_latent), int(d_v), _ptr(o_lat),
+                                 int(o_lat.stride(0)), _ptr(w_uv), _dt(w_uv), _ptr(out), int(out.stride(0)),
+                                 _dt(out), _stream(stream)), "kdv_unabsorb_o")
 
 
 def kdv_combine(o_part: torch.Tensor, lse_part: torch.Tensor, S: int, rows: int, d: int,

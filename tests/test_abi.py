@@ -183,3 +183,18 @@ def test_library_has_no_oracle_dependency():
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, fn
                 assert "kdv_oracle" not in txt, fn
+
+
+def test_projection_validation(lib):
+    fa, fu = lib.kdv_absorb_q, lib.kdv_unabsorb_o
+    B, F = kdv.KDV_BF16, kdv.KDV_F32
+    # rows not a multiple of H; null pointers; strides shorter than rows; dtypes; limits
+    assert fa(13, 4, 512, 128, 0x1000, 128, B, 0x2000, B, 0x3000, 576, B, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fa(16, 4, 512, 128, None, 128, B, 0x2000, B, 0x3000, 576, B, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fa(16, 4, 512, 128, 0x1000, 100, B, 0x2000, B, 0x3000, 576, B, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fa(16, 4, 512, 128, 0x1000, 128, 9, 0x2000, B, 0x3000, 576, B, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fa(16, 4, 512, 600, 0x1000, 600, B, 0x2000, B, 0x3000, 576, B, None) == kdv.KDV_ERR_UNSUPPORTED
+    assert fa(0, 4, 512, 128, None, 128, B, None, B, None, 576, B, None) == kdv.KDV_OK
+    assert fu(13, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fu(16, 4, 513, 128, 0x1000, 513, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_UNSUPPORTED
+    assert fu(16, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 100, F, None) == kdv.KDV_ERR_INVALID_ARG

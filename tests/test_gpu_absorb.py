@@ -1,0 +1,117 @@
+"""GPU parity of kdv_absorb_q / kdv_unabsorb_o against the oracle, and the
+whole absorbed layer (absorb -> verify -> up-project) against the oracle's
+non-absorbed MLA.
+
+The projections are the latent projection the verify kernel absorbs (page
+"The Architecture of Diagnosis", section "Phase 1: Custom CUDA Kernels",
+item 2). Accumulation is fp32 on both GPU kernels, so fp32 outputs are held to
+a relative 2e-5; bf16 outputs to one bf16 unit in the last place.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from speculative_tree_verify_mla_b200 import datagen, kdv
+from tests.parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+
+
+def _t(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dtype).to(dev)
+
+
+def _rel_err(got, want):
+    return np.abs(got - want).max() / np.abs(want).max()
+
+
+@pytest.mark.parametrize("T,wdt", [(13, torch.bfloat16), (1, torch.bfloat16), (40, torch.bfloat16),
+                                   (13, torch.float32)])
+def test_absorb_q_kimi(T, wdt):
+    case = datagen.kimi_layer_case(L=64, T=T, seed=5)
+    q_nope, w_uk, _ = datagen.layer_weights(case)
+    ref = oracle.absorb_q(case.H, q_nope, w_uk)
+    out = torch.full((case.rows, 512), float("nan"), device=dev)
+    kdv.kdv_absorb_q(case.H, _t(q_nope, wdt), _t(w_uk, wdt), out)
+    torch.cuda.synchronize()
+    assert _rel_err(out.cpu().numpy(), ref) < 2e-5
+
+
+def test_absorb_q_into_verify_rows_bf16():
+    """q_lat written as bf16 straight into the first 512 columns of 576-wide
+    q rows; the q_rope columns stay untouched."""
+    case = datagen.kimi_layer_case(L=64, T=13, seed=6)
+    q_nope, w_uk, _ = datagen.layer_weights(case)
+    ref = oracle.absorb_q(case.H, q_nope, w_uk)
+    q = torch.full((case.rows, 576), 3.0, dtype=torch.bfloat16, device=dev)
+    kdv.kdv_absorb_q(case.H, _t(q_nope, torch.bfloat16), _t(w_uk, torch.bfloat16), q[:, :512])
+    torch.cuda.synchronize()
+    got = q.float().cpu().numpy()
+    assert np.all(got[:, 512:] == 3.0)
+    # round-to-nearest-even of the fp32 sum: within one bf16 ulp of the exact
+    # value, plus the fp32 accumulation error of a 128-term sum (for entries
+    # near zero, where one ulp is tiny)
+    assert np.all(np.abs(got[:, :512] - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-6)
+
+
+@pytest.mark.parametrize("T,out_dt", [(13, torch.float32), (40, torch.float32), (13, torch.bfloat16)])
+def test_unabsorb_o_kimi(T, out_dt):
+    case = datagen.kimi_layer_case(L=64, T=T, seed=7)
+    _, _, w_uv = datagen.layer_weights(case)
+    o_lat = np.random.default_rng(T).standard_normal((case.rows, 512)).astype(np.float32) * 0.05
+    ref = oracle.unabsorb_o(case.H, o_lat, w_uv)
+    out = torch.full((case.rows, 128), float("nan"), dtype=out_dt, device=dev)
+    kdv.kdv_unabsorb_o(case.H, _t(o_lat), _t(w_uv, torch.bfloat16), out)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    if out_dt == torch.float32:
+        assert _rel_err(got, ref) < 2e-5
+    else:
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-6)
+
+
+def test_tiny_layer_end_to_end_fp32():
+    """The tiny fp32 layer through the GPU: absorb, verify (SIMT), up-project,
+    against the oracle's non-absorbed MLA (explicit K = c_kv W_UK, V = c_kv W_UV)."""
+    case = datagen.tiny_fp32_case()
+    q_nope, w_uk, w_uv = datagen.tiny_fp32_layer(case)
+    D_c, D_r, H = case.D_c, case.D_r, case.H
+    L, T = int(case.prefix_len[0]), int(case.tree_T[0])
+    out_ref, lse_ref = oracle.verify_mla(H=H, L=L, parent=case.parent, D_c=D_c, D_r=D_r, D_n=case.D_n,
+                                         D_v=case.D_v, scale=case.scale, q_nope=q_nope,
+                                         q_rope=case.q[:, D_c:], c_kv=case.kv[:, :D_c],
+                                         k_rope=case.kv[:, D_c:], w_uk=w_uk, w_uv=w_uv)
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_SIMT, num_splits=2)
+    dc.q[:, :D_c] = float("nan")                           # the absorb must fill these
+    kdv.kdv_absorb_q(H, _t(q_nope), _t(w_uk), dc.q[:, :D_c])
+    dc.run()
+    out = torch.empty(case.rows, case.D_v, device=dev)
+    kdv.kdv_unabsorb_o(H, dc.o, _t(w_uv), out)
+    torch.cuda.synchronize()
+    assert dc.error_flag() == 0
+    np.testing.assert_allclose(out.cpu().numpy(), out_ref, rtol=2e-5, atol=2e-6)
+    np.testing.assert_allclose(dc.lse.cpu().numpy(), lse_ref, rtol=2e-5, atol=2e-6)
+
+
+def test_kimi_layer_end_to_end_bf16():
+    """Kimi shape at L=1500: bf16 absorb into the q rows, the tensor-core
+    verify, fp32 up-projection; against the non-absorbed fp64 oracle. The GPU
+    rounds q_lat to bf16 and P to bf16, so the attention bars apply."""
+    case = datagen.kimi_layer_case(L=1500, T=13, seed=8)
+    q_nope, w_uk, w_uv = datagen.layer_weights(case)
+    L, T = 1500, 13
+    out_ref, lse_ref = oracle.verify_mla(H=64, L=L, parent=case.parent, D_c=512, D_r=64, D_n=128,
+                                         D_v=128, scale=case.scale, q_nope=q_nope,
+                                         q_rope=case.q[:, 512:], c_kv=case.kv[:, :512],
+                                         k_rope=case.kv[:, 512:], w_uk=w_uk, w_uv=w_uv)
+    dc = kdv.DeviceCase(case, num_splits=0)
+    kdv.kdv_absorb_q(64, _t(q_nope, torch.bfloat16), _t(w_uk, torch.bfloat16), dc.q[:, :512])
+    dc.run()
+    out = torch.empty(case.rows, 128, device=dev)
+    kdv.kdv_unabsorb_o(64, dc.o, _t(w_uv, torch.bfloat16), out)
+    torch.cuda.synchronize()
+    assert dc.error_flag() == 0
+    assert_parity(out.cpu().numpy(), dc.lse.cpu().numpy(), out_ref, lse_ref,
+                  max_tol=float("inf"), mean_tol=float("inf"), lse_tol=5e-3)
