@@ -75,6 +75,10 @@ def _load():
             lib.oracle_tree_accept.restype = c.c_int
             lib.oracle_accept_commit.argtypes = [c.c_int32, c.c_int32, c.c_int32, _i32p, _i32p]
             lib.oracle_accept_commit.restype = None
+            _f32p_ = _f32p
+            lib.oracle_tree_build.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int32, _i32p, _f32p_,
+                                              _i32p, _i32p, _i32p, _f32p_]
+            lib.oracle_tree_build.restype = c.c_int
             _lib = lib
     return _lib
 
@@ -276,3 +280,28 @@ def accept_case(case):
     if pt is not None:
         out["page_table"] = pt
     return out
+
+
+# ---------------------------------------------------------------------------
+# Best-first draft-tree construction (kdv_oracle.cpp: "Best-first draft-tree
+# construction"; page "The Architecture of Diagnosis", section "Phase 1:
+# Custom CUDA Kernels", item 1).
+
+def tree_build(T: int, root_token: int, cand_token, cand_logp):
+    """First T nodes in (score desc, candidate path asc) order.
+
+    cand_token int32 [D][K], cand_logp float32 [D][K] (log-probabilities).
+    Returns (parent, token, depth, score) of the emitted nodes.
+    """
+    ct = np.ascontiguousarray(cand_token, dtype=np.int32)
+    cl = np.ascontiguousarray(cand_logp, dtype=np.float32)
+    D, K = ct.shape
+    parent = np.zeros(T, dtype=np.int32)
+    token = np.zeros(T, dtype=np.int32)
+    depth = np.zeros(T, dtype=np.int32)
+    score = np.zeros(T, dtype=np.float32)
+    n = _load().oracle_tree_build(int(T), int(D), int(K), int(root_token), ct, cl, parent, token, depth,
+                                  score)
+    if n < 0:
+        raise ValueError("bad sizes")
+    return parent[:n], token[:n], depth[:n], score[:n]

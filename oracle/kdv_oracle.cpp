@@ -374,3 +374,70 @@ void oracle_accept_commit(int32_t L, int32_t T, int32_t len, const int32_t* path
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Best-first draft-tree construction (page "The Architecture of Diagnosis",
+// section "Phase 1: Custom CUDA Kernels", item 1: a GPU-resident builder
+// replaces a host heap that grows the draft tree best-first). The page gives
+// no scoring; the reading used here follows a block drafter that proposes K
+// candidate tokens with log-probabilities for each of D future positions:
+//
+//   node   = root (depth 0, the last committed token) or a path of candidate
+//            choices (j_1, ..., j_d), one per position 1..d (depth d <= D)
+//   score  = fp32 sum of logp[i-1][j_i] along the path, accumulated root-first
+//            (child = parent + logp, one float add)
+//   order  = score descending, ties by the path compared digit by digit
+//            (a prefix first, then the smaller candidate index)
+//   tree   = the first T nodes in that order, emitted in that order with
+//            parent = output index of the node's parent (-1 for the root).
+// With every logp <= 0 a node never outranks its parent, so this is exactly
+// what a best-first expansion (pop the best frontier node, push its K
+// children) emits. Done here as that expansion with a linear frontier scan.
+
+namespace {
+struct Cand { float score; uint64_t key; int32_t depth, parent, token; bool live; };
+// true when a ranks before b
+bool cand_before(const Cand& a, const Cand& b) {
+  if (a.score != b.score) return a.score > b.score;
+  return a.key < b.key;
+}
+}  // namespace
+
+extern "C" {
+
+// Returns the number of nodes emitted (T unless the candidates run out first),
+// or -1 on bad sizes (T < 1, D > 16, K > 8).
+int oracle_tree_build(int32_t T, int32_t D, int32_t K, int32_t root_token, const int32_t* cand_token,
+                      const float* cand_logp, int32_t* parent, int32_t* token, int32_t* depth, float* score) {
+  if (T < 1 || D < 0 || D > 16 || K < 1 || K > 8) return -1;
+  std::vector<Cand> f;
+  f.push_back(Cand{0.0f, 0u, 0, -1, root_token, true});
+  int32_t n = 0;
+  for (; n < T; ++n) {
+    int best = -1;
+    for (int i = 0; i < (int)f.size(); ++i)
+      if (f[i].live && (best < 0 || cand_before(f[i], f[best]))) best = i;
+    if (best < 0) break;
+    Cand c = f[best];
+    f[best].live = false;
+    parent[n] = c.parent;
+    token[n] = c.token;
+    depth[n] = c.depth;
+    score[n] = c.score;
+    if (c.depth < D) {
+      for (int32_t j = 0; j < K; ++j) {
+        const float lp = cand_logp[(int64_t)c.depth * K + j];
+        const float s = c.score + lp;
+        // the path as D base-(K+1) digits, most significant first, 0 past
+        // the end: numeric order = digit-by-digit order with a prefix first
+        uint64_t place = 1;
+        for (int32_t e = c.depth + 1; e < D; ++e) place *= (uint64_t)(K + 1);
+        const uint64_t key = c.key + (uint64_t)(j + 1) * place;
+        f.push_back(Cand{s, key, c.depth + 1, n, cand_token[(int64_t)c.depth * K + j], true});
+      }
+    }
+  }
+  return n;
+}
+
+}  // extern "C"
