@@ -376,6 +376,47 @@ def time_tree_accept(dev, stream, peaks, n_bufs: int = 40, reps: int = 20):
             "timing": f"{n_bufs} distinct logits buffers ({n_bufs * bytes_ / 1e6:.0f} MB > L2), graph replay"}
 
 
+def time_projections(dev, stream, peaks, n_layers: int = 61, reps: int = 10):
+    """q_lat = W_UK q_nope and out = W_UV^T o_lat for the Kimi-shape layer
+    (H=64, 512/128/128, T=13): n_layers distinct bf16 weight sets (n_layers x
+    16.8 MB > L2), graph-replayed; HBM-bound on the weights."""
+    import torch
+    from speculative_tree_verify_mla_b200 import datagen, kdv
+    case = datagen.kimi_layer_case(L=16, T=T_TREE, seed=1)
+    q_nope, w_uk, w_uv = datagen.layer_weights(case)
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).to(dev)
+    qn = bf(q_nope)
+    wk0, wv0 = bf(w_uk), bf(w_uv)
+    wks = [wk0] + [wk0.clone() for _ in range(n_layers - 1)]
+    wvs = [wv0] + [wv0.clone() for _ in range(n_layers - 1)]
+    q = torch.zeros(case.rows, 576, dtype=torch.bfloat16, device=dev)
+    o_lat = torch.randn(case.rows, 512, device=dev) * 0.05
+    out = torch.empty(case.rows, 128, device=dev)
+
+    def absorb(s):
+        for wk in wks:
+            kdv.kdv_absorb_q(case.H, qn, wk, q[:, :512], s)
+
+    def unabsorb(s):
+        for wv in wvs:
+            kdv.kdv_unabsorb_o(case.H, o_lat, wv, out, s)
+
+    res = {}
+    for name, fn, wbytes in (("absorb_q", absorb, wk0.numel() * 2), ("unabsorb_o", unabsorb, wv0.numel() * 2)):
+        with torch.cuda.stream(stream):
+            fn(stream)
+        stream.synchronize()
+        g = graph_of(fn, stream)
+        us = replay_us(g, stream, reps) / n_layers
+        del g
+        gbs = wbytes / (us * 1e-6) / 1e9
+        res[name] = {"us_per_layer": us, "weight_bytes": wbytes, "achieved_gbs": gbs,
+                     "frac": gbs / peaks["hbm_gbs"]}
+    res.update({"bound": "hbm", "peak_gbs": peaks["hbm_gbs"], "workload": f"kimi_proj_T{T_TREE}",
+                "timing": f"{n_layers} distinct weight sets ({n_layers * 16.8:.0f} MB > L2), graph replay"})
+    return res
+
+
 def run_gpu(args):
     import torch
     from speculative_tree_verify_mla_b200 import kdv
@@ -544,6 +585,7 @@ def run_gpu(args):
 
     if args.workload == "kimi" and rank == 0:
         result["tree_accept"] = time_tree_accept(dev, stream, peaks)
+        result["projections"] = time_projections(dev, stream, peaks)
 
     # ---- CPU oracle on the host cores (rank 0, N=1 only): baseline + spot parity ----
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -66,6 +66,8 @@ typedef enum {
 #define KDV_DERR_BAD_TOKEN 4   /* tree-accept: token id out of range        */
 #define KDV_DERR_TIMEOUT 5     /* a bounded in-kernel wait ran out (~1 s);
                                   the kernel stopped early, output invalid  */
+#define KDV_DERR_BAD_SCORE 6   /* tree build: a NaN candidate log-probability
+                                  (read as -inf)                            */
 
 /* Element type of q and kv. */
 #define KDV_BF16 0
@@ -296,6 +298,39 @@ KDV_API kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_laten
 KDV_API kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v,
                                   const float* o_lat, int64_t o_lat_stride, const void* w_uv, int32_t w_dtype,
                                   void* out, int64_t out_stride, int32_t out_dtype, void* stream);
+
+/*
+ * kdv_tree_build -- best-first draft-tree construction on the device (the
+ * GPU-resident builder of page "The Architecture of Diagnosis", section
+ * "Phase 1: Custom CUDA Kernels", item 1, which replaces a host heap). The
+ * page gives no scoring; this library reads it as: a block drafter proposes,
+ * for each of D future positions, K candidate tokens with log-probabilities;
+ * a node is a path of candidate choices (one per position, root = the last
+ * committed token at depth 0); its score is the fp32 sum of the chosen
+ * log-probabilities, added root first; the tree of request b is the first
+ * T_b nodes in (score descending, path ascending digit by digit with a prefix
+ * first) order, emitted in that order -- parents precede children, so the
+ * output feeds kdv_tree_mask_build directly. With log-probabilities <= 0 this
+ * equals the best-first expansion. A NaN log-probability is read as -inf and
+ * reported (KDV_DERR_BAD_SCORE). A budget above the number of paths is
+ * reported (KDV_DERR_BAD_LENGTH); the missing nodes get parent -1, token -1.
+ */
+typedef struct kdv_tree_build_params {
+  int32_t batch;              /* B in [1, KDV_MAX_BATCH]                           */
+  int32_t max_T;              /* [1, 64]: bound on every budget T_b                 */
+  int32_t depth;              /* D in [0, 16]: draft positions with candidates      */
+  int32_t topk;               /* K in [1, 8]: candidates per position               */
+  const int32_t* tree_off;    /* [B+1] device: T_b = tree_off[b+1] - tree_off[b]    */
+  const int32_t* root_token;  /* [B] token of each root                             */
+  const int32_t* cand_token;  /* [B][D][K] candidate tokens                          */
+  const float* cand_logp;     /* [B][D][K] their log-probabilities                   */
+  int32_t* parent;            /* [sumT] out: request-local parent index, -1 = root   */
+  int32_t* token;             /* [sumT] out                                          */
+  int32_t* depth_out;         /* [sumT] out, nullable                                */
+  float* score;               /* [sumT] out, nullable                                */
+  int32_t* d_err;             /* nullable device error flag                          */
+} kdv_tree_build_params;
+KDV_API kdv_status kdv_tree_build(const kdv_tree_build_params* p, void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,7 +39,7 @@ import numpy as np
 _IDS = {
     "tree": 1, "ckv": 2, "krope": 3, "qlat": 4, "qrope": 5, "qnope": 6,
     "wuk": 7, "wuv": 8, "prefix": 9, "treeT": 10, "perm": 11, "tokens": 12,
-    "logits": 13, "misc": 14,
+    "logits": 13, "misc": 14, "cands": 15,
 }
 
 
@@ -390,3 +390,54 @@ def batched_accept_case(B: int = 8, seed: int = 4, vocab: int = KIMI_VOCAB) -> A
     parents = [random_tree(int(tT[b]), rng_for(seed, "tree", b, int(tT[b]))) for b in range(B)]
     return make_accept_case(f"paged_accept_B{B}", parents=parents, vocab=vocab, seed=seed,
                             prefix_len=[int(x) for x in plen], paged=True)
+
+
+
+# ---------------------------------------------------------------------------
+# Draft-tree construction inputs: a block drafter's per-position candidates.
+#
+# The pages name a block size of 16 and a node budget of 32 for the drafter
+# (page "The Three Acts of Engineering", section "Act III", "The Reproducible
+# Estimator"); a block of 16 positions after the root gives D = 15 draft
+# positions here. K = 8 candidates per position is this library's choice (the
+# builder's limit).
+
+@dataclasses.dataclass
+class BuildCase:
+    """Per request: root token, K candidate tokens and log-probabilities for
+    each of D positions, and the node budget (tree_off CSR)."""
+    depth: int
+    topk: int
+    tree_off: np.ndarray        # int32 [B+1]
+    root_token: np.ndarray      # int32 [B]
+    cand_token: np.ndarray      # int32 [B][D][K]
+    cand_logp: np.ndarray       # float32 [B][D][K]
+
+    @property
+    def batch(self) -> int:
+        return int(self.tree_off.shape[0] - 1)
+
+
+def make_build_case(budgets: List[int], D: int = 15, K: int = 8, seed: int = 0,
+                    vocab: int = KIMI_VOCAB, quantised: bool = False) -> BuildCase:
+    """Candidates: per position, K distinct random tokens whose log-probabilities
+    are the K largest entries of a log-softmax over K+8 N(0, 2) logits (sorted
+    descending). ``quantised`` rounds them to multiples of 1/4 so that score
+    ties are common."""
+    B = len(budgets)
+    rng = rng_for(seed, "cands", B, D, K)
+    toks = np.zeros((B, D, K), dtype=np.int32)
+    logp = np.zeros((B, D, K), dtype=np.float32)
+    for b in range(B):
+        for d in range(D):
+            toks[b, d] = rng.choice(vocab, size=K, replace=False)
+            z = rng.standard_normal(K + 8) * 2.0
+            ls = z - (np.log(np.exp(z - z.max()).sum()) + z.max())
+            top = np.sort(ls)[::-1][:K]
+            if quantised:
+                top = np.round(top * 4) / 4
+            logp[b, d] = top.astype(np.float32)
+    off = np.zeros(B + 1, dtype=np.int32)
+    off[1:] = np.cumsum(budgets)
+    root = rng.integers(0, vocab, size=B).astype(np.int32)
+    return BuildCase(depth=D, topk=K, tree_off=off, root_token=root, cand_token=toks, cand_logp=logp)

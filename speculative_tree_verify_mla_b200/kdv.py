@@ -29,6 +29,7 @@ KDV_DERR_BAD_SLOT = 2
 KDV_DERR_BAD_LENGTH = 3
 KDV_DERR_BAD_TOKEN = 4
 KDV_DERR_TIMEOUT = 5
+KDV_DERR_BAD_SCORE = 6
 
 KDV_BF16 = 0
 KDV_F32 = 1
@@ -43,7 +44,7 @@ KDV_MAX_BATCH = 128
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
             "kdv_verify_attn_noalloc", "kdv_combine", "kdv_tree_accept_workspace",
-            "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o")
+            "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o", "kdv_tree_build")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -91,6 +92,17 @@ class AcceptParams(ctypes.Structure):
     ]
 
 
+class BuildParams(ctypes.Structure):
+    """Mirror of ``kdv_tree_build_params`` (field order and types must match kdv.h)."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("max_T", ctypes.c_int32), ("depth", ctypes.c_int32),
+        ("topk", ctypes.c_int32), ("tree_off", ctypes.c_void_p), ("root_token", ctypes.c_void_p),
+        ("cand_token", ctypes.c_void_p), ("cand_logp", ctypes.c_void_p),
+        ("parent", ctypes.c_void_p), ("token", ctypes.c_void_p), ("depth_out", ctypes.c_void_p),
+        ("score", ctypes.c_void_p), ("d_err", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -132,6 +144,8 @@ def load() -> ctypes.CDLL:
         lib.kdv_unabsorb_o.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int32, c.c_void_p, c.c_int64,
                                        c.c_void_p, c.c_int32, c.c_void_p, c.c_int64, c.c_int32, c.c_void_p]
         lib.kdv_unabsorb_o.restype = c.c_int
+        lib.kdv_tree_build.argtypes = [c.POINTER(BuildParams), c.c_void_p]
+        lib.kdv_tree_build.restype = c.c_int
         _lib = lib
     return _lib
 
@@ -346,6 +360,17 @@ def make_accept_params(**kw) -> AcceptParams:
             setattr(p, k, int(v.data_ptr()))
         else:
             setattr(p, k, v)
+    return p
+
+
+def kdv_tree_build(params: BuildParams, stream=None) -> None:
+    _check(load().kdv_tree_build(ctypes.byref(params), _stream(stream)), "kdv_tree_build")
+
+
+def make_build_params(**kw) -> BuildParams:
+    p = BuildParams()
+    for k, v in kw.items():
+        setattr(p, k, int(v.data_ptr()) if isinstance(v, torch.Tensor) else v)
     return p
 
 

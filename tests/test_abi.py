@@ -42,7 +42,8 @@ def test_status_strings(lib):
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
-                                       (kdv.AcceptParams, "kdv_accept_params")])
+                                       (kdv.AcceptParams, "kdv_accept_params"),
+                                       (kdv.BuildParams, "kdv_tree_build_params")])
 def test_params_struct_layout(tmp_path, cls, cname):
     """ctypes mirror matches the C struct: compile a probe against kdv.h."""
     fields = [f[0] for f in cls._fields_]
@@ -198,3 +199,21 @@ def test_projection_validation(lib):
     assert fu(13, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_INVALID_ARG
     assert fu(16, 4, 513, 128, 0x1000, 513, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_UNSUPPORTED
     assert fu(16, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 100, F, None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_tree_build_validation(lib):
+    def bp(**over):
+        base = dict(batch=2, max_T=32, depth=15, topk=8, tree_off=0x1000, root_token=0x2000,
+                    cand_token=0x3000, cand_logp=0x4000, parent=0x5000, token=0x6000, depth_out=None,
+                    score=None, d_err=None)
+        base.update(over)
+        return kdv.make_build_params(**base)
+    f = lambda **o: lib.kdv_tree_build(ctypes.byref(bp(**o)), None)
+    assert f(batch=0) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(max_T=65) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(depth=17) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(topk=9) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(topk=0) == kdv.KDV_ERR_UNSUPPORTED
+    assert f(parent=None) == kdv.KDV_ERR_INVALID_ARG
+    assert f(cand_logp=None) == kdv.KDV_ERR_INVALID_ARG
+    assert lib.kdv_tree_build(None, None) == kdv.KDV_ERR_INVALID_ARG

@@ -96,3 +96,16 @@ def test_build_rejects_bad_sizes():
         oracle.tree_build(0, 1, np.zeros((2, 2), np.int32), np.zeros((2, 2), np.float32))
     with pytest.raises(ValueError):
         oracle.tree_build(4, 1, np.zeros((2, 9), np.int32), np.zeros((2, 9), np.float32))
+
+
+def test_build_nan_logprob_reads_as_minus_inf():
+    rng = np.random.default_rng(4)
+    cand_logp = np.log(rng.dirichlet(np.ones(3), size=3)).astype(np.float32)
+    cand_token = rng.integers(0, 9, size=(3, 3)).astype(np.int32)
+    with_nan = cand_logp.copy()
+    with_nan[1, 0] = np.nan
+    with_inf = cand_logp.copy()
+    with_inf[1, 0] = -np.inf
+    a = oracle.tree_build(30, 5, cand_token, with_nan)
+    b = _brute_force(30, 5, cand_token, with_inf)
+    assert list(a[0]) == b[0] and list(a[1]) == b[1]
