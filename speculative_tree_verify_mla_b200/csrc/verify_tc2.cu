@@ -66,9 +66,9 @@ constexpr int KV_STAGES = 4;
 constexpr int KV_STAGE_BYTES = STAGE_BLOCKS * KBLOCK_BYTES;   // 48 KB
 constexpr int Q_STAGES = 3;                         // ring stages covering q_lat staging
 constexpr int STAGES_PER_TILE = QK_BLOCKS / STAGE_BLOCKS;
-constexpr int V_STAGES = 8;
+constexpr int V_STAGES = 6;
 constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
-constexpr int NP = 2;
+constexpr int NP = 3;                               // P slots per O CTA
 constexpr int P_BYTES = ROWS * KEYS * 2;
 constexpr int P_KCHUNK_BYTES = ROWS * 16;           // 8 keys of all 128 rows (interleaved core matrices)
 constexpr int P_MSG_BYTES = P_BYTES + ROWS * 4;
@@ -88,7 +88,7 @@ static_assert(Q_STAGES < KV_STAGES, "ring too small");
 // Shared-memory layout (same offsets in all four CTAs; mapa() relies on it).
 //   S CTAs: [0, 196608) KV ring (4 x 48 KB; q_lat staging in the first 128 KB
 //           at start-up); [196608, 212992) q_rope; row-max / row-sum exchange.
-//   O CTAs: [0, 131072) V ring (8 x 16 KB); P slots; final stats.
+//   O CTAs: [0, 98304) V ring (6 x 16 KB); 3 P slots; final stats.
 constexpr int OFF_RING = 0;
 constexpr int OFF_QROPE = KV_STAGES * KV_STAGE_BYTES;
 constexpr int OFF_XCHG = OFF_QROPE + QBLOCK_BYTES;           // float [2][2][128] + [128] (S side)
@@ -109,11 +109,13 @@ static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of shared memory");
 // Barrier slots (each CTA initialises the slots its role uses).
 // S pair. KV_FULL, S_EMPTY, QROPE_FULL and Q_READY are used in CTA 0 only
 // (the MMA issuer's barriers); the others in both S CTAs.
-constexpr int B_KV_FULL = 0, B_KV_EMPTY = 4, B_S_FULL = 8, B_S_EMPTY = 9, B_P_EMPTY = 10,
-              B_QLAT_FULL = 12, B_QROPE_FULL = 13, B_Q_READY = 14, B_S_DRAIN = 15;
+constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + KV_STAGES, B_S_FULL = B_KV_EMPTY + KV_STAGES,
+              B_S_EMPTY = B_S_FULL + 1, B_P_EMPTY = B_S_EMPTY + 1, B_QLAT_FULL = B_P_EMPTY + NP,
+              B_QROPE_FULL = B_QLAT_FULL + 1, B_Q_READY = B_QROPE_FULL + 1, B_S_DRAIN = B_Q_READY + 1;
 // O pair. V_FULL, READY and O_DRAIN in CTA 2 only.
-constexpr int B_V_FULL = 16, B_V_EMPTY = 24, B_P_FULL = 32, B_READY = 34, B_PV_DONE = 36,
-              B_STATS = 38, B_O_DRAIN = 39;
+constexpr int B_V_FULL = B_S_DRAIN + 1, B_V_EMPTY = B_V_FULL + V_STAGES, B_P_FULL = B_V_EMPTY + V_STAGES,
+              B_READY = B_P_FULL + NP, B_PV_DONE = B_READY + NP, B_STATS = B_PV_DONE + NP,
+              B_O_DRAIN = B_STATS + 1;
 static_assert(B_O_DRAIN < NUM_BARS, "barrier slots");
 
 constexpr uint16_t S_PAIR = 0x3, O_PAIR = 0xC;     // cluster CTA masks
@@ -425,8 +427,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const float sl2 = a.scale * LOG2E;
       float m_run = -INFINITY, l_part = 0.f;
       const uint32_t o_rank = 2 + half;                       // this CTA's O partner
-      const uint32_t pslot = mapa(base + OFF_P, o_rank) + hw * P_SLOT_BYTES;
-      const uint32_t pbar = mapa(c.bar(B_P_FULL), o_rank) + hw * 8;
+      const uint32_t pslot0 = mapa(base + OFF_P, o_rank);
+      const uint32_t pbar0 = mapa(c.bar(B_P_FULL), o_rank);
       for (int i = 0; i < n_stiles; ++i) {
         ok = wait_warp(c, c.bar(B_S_FULL), i & 1) && ok;
         const bool wok = __all_sync(0xffffffffu, ok);
@@ -434,11 +436,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         if (wok) {
           __syncwarp();
           tc_fence_after();
-          const uint32_t sa = tmem + lane_base + TMEM_S_COL + hw * KEYS;
-          tmem_ld32(sa, *reinterpret_cast<uint32_t(*)[32]>(sv));
-          tmem_ld32(sa + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-          tmem_ld32(sa + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
-          tmem_ld32(sa + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+          // one 128-column load: the S half arrives in a single TMEM round trip
+          tmem_ld128(tmem + lane_base + TMEM_S_COL + hw * KEYS, sv);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
@@ -482,8 +481,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           m_run = m_tile;
         }
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        // P tile 2i + hw goes to O-side slot hw
-        ok = wait_warp(c, c.bar(B_P_EMPTY + hw), (i & 1) ^ 1) && ok;
+        // P tile pt = 2i + hw goes to O-side slot pt % NP (the O side
+        // consumes P tiles in order, slot by slot)
+        const int pt = 2 * i + hw, pslot_i = pt % NP;
+        const uint32_t pslot = pslot0 + pslot_i * P_SLOT_BYTES;
+        const uint32_t pbar = pbar0 + pslot_i * 8;
+        ok = wait_warp(c, c.bar(B_P_EMPTY + pslot_i), ((pt / NP) & 1) ^ 1) && ok;
         float lsum = 0.f;
 #pragma unroll
         for (int ch = 0; ch < KEYS / 8; ++ch) {
