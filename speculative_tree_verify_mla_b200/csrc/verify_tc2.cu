@@ -424,6 +424,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         if (lane == 0) arrive_on(c.bar(B_Q_READY), lead_rank, rank);
       }
       const uint64_t mask_t = valid ? a.mask[p.tree_base[b] + row / H] : 0ull;
+      // a warp whose 32 rows all lie past the request's last row (the tail
+      // of its last row tile) sends zeros and does no softmax work
+      const bool warp_rows = __any_sync(0xffffffffu, valid);
       const float sl2 = a.scale * LOG2E;
       float m_run = -INFINITY, l_part = 0.f;
       const uint32_t o_rank = 2 + half;                       // this CTA's O partner
@@ -456,12 +459,27 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             sv[k] = __float_as_uint(xk);
             m_half = fmaxf(m_half, xk);
           }
-        } else {
+        } else if (warp_rows) {
+          // visibility of the tile's 128 keys as four 32-bit words: prefix
+          // keys (j < L) inside the split, tree keys j = L+u with bit u of
+          // the row's ancestor mask, nothing at or past the split's end
+          const int n_pre = max(0, min(KEYS, min(L, k_hi) - key0));
+          const int n_lim = max(0, min(KEYS, k_hi - key0));
+          uint32_t vw[KEYS / 32];
+#pragma unroll
+          for (int w = 0; w < KEYS / 32; ++w) {
+            const int lo = 32 * w;
+            const uint32_t pre = n_pre >= lo + 32 ? 0xffffffffu : (n_pre <= lo ? 0u : (1u << (n_pre - lo)) - 1u);
+            const uint32_t lim = n_lim >= lo + 32 ? 0xffffffffu : (n_lim <= lo ? 0u : (1u << (n_lim - lo)) - 1u);
+            const int sft = key0 + lo - L;              // tree index of the word's first key
+            uint32_t tree = 0u;
+            if (sft >= 0 && sft < 64) tree = (uint32_t)(mask_t >> sft);
+            else if (sft < 0 && sft > -32) tree = (uint32_t)(mask_t << (-sft));
+            vw[w] = valid ? ((pre | tree) & lim) : 0u;
+          }
 #pragma unroll
           for (int k = 0; k < KEYS; ++k) {
-            const int j = key0 + k;
-            bool vis = valid && j < k_hi;
-            if (j >= L) vis = vis && ((mask_t >> ((j - L) & 63)) & 1ull);
+            const bool vis = (vw[k >> 5] >> (k & 31)) & 1u;
             const float xk = vis ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
             sv[k] = __float_as_uint(xk);
             m_half = fmaxf(m_half, xk);
@@ -488,19 +506,24 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const uint32_t pbar = pbar0 + pslot_i * 8;
         ok = wait_warp(c, c.bar(B_P_EMPTY + pslot_i), ((pt / NP) & 1) ^ 1) && ok;
         float lsum = 0.f;
+        if (warp_rows) {
 #pragma unroll
-        for (int ch = 0; ch < KEYS / 8; ++ch) {
-          uint32_t w[4];
+          for (int ch = 0; ch < KEYS / 8; ++ch) {
+            uint32_t w[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float p0 = ex2(__uint_as_float(sv[8 * ch + 2 * q]) - m_use);
-            const float p1 = ex2(__uint_as_float(sv[8 * ch + 2 * q + 1]) - m_use);
-            lsum += p0 + p1;
-            w[q] = pack_bf16x2(p0, p1);
+            for (int q = 0; q < 4; ++q) {
+              const float p0 = ex2(__uint_as_float(sv[8 * ch + 2 * q]) - m_use);
+              const float p1 = ex2(__uint_as_float(sv[8 * ch + 2 * q + 1]) - m_use);
+              lsum += p0 + p1;
+              w[q] = pack_bf16x2(p0, p1);
+            }
+            // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
+            // so a warp's 32 rows fill 512 contiguous bytes per store
+            if (ok) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, w[0], w[1], w[2], w[3], pbar);
           }
-          // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
-          // so a warp's 32 rows fill 512 contiguous bytes per store
-          if (ok) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, w[0], w[1], w[2], w[3], pbar);
+        } else if (ok) {
+#pragma unroll 1
+          for (int ch = 0; ch < KEYS / 8; ++ch) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, 0u, 0u, 0u, 0u, pbar);
         }
         l_part += lsum;
         // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
