@@ -390,11 +390,26 @@ verify_tc_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
             m_tile = fmaxf(m_tile, xk);
           }
         } else {
+          // visibility of the tile's keys as 32-bit words: prefix keys
+          // inside the split, tree keys L+u with bit u of the row's ancestor
+          // mask, nothing at or past the split's end (keeps S in registers)
+          const int n_pre = max(0, min(KEYS, min(L, k_hi) - key0));
+          const int n_lim = max(0, min(KEYS, k_hi - key0));
+          uint32_t vw[KEYS / 32];
+#pragma unroll
+          for (int w = 0; w < KEYS / 32; ++w) {
+            const int lo = 32 * w;
+            const uint32_t pre = n_pre >= lo + 32 ? 0xffffffffu : (n_pre <= lo ? 0u : (1u << (n_pre - lo)) - 1u);
+            const uint32_t lim = n_lim >= lo + 32 ? 0xffffffffu : (n_lim <= lo ? 0u : (1u << (n_lim - lo)) - 1u);
+            const int sft = key0 + lo - L;
+            uint32_t tree = 0u;
+            if (sft >= 0 && sft < 64) tree = (uint32_t)(mask_t >> sft);
+            else if (sft < 0 && sft > -32) tree = (uint32_t)(mask_t << (-sft));
+            vw[w] = valid ? ((pre | tree) & lim) : 0u;
+          }
 #pragma unroll
           for (int k = 0; k < KEYS; ++k) {
-            const int j = key0 + k;
-            bool vis = valid && j < k_hi;
-            if (j >= L) vis = vis && ((mask_t >> ((j - L) & 63)) & 1ull);
+            const bool vis = (vw[k >> 5] >> (k & 31)) & 1u;
             const float xk = vis ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
             sv[k] = __float_as_uint(xk);
             m_tile = fmaxf(m_tile, xk);
