@@ -186,6 +186,24 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's x (device time of the slowest rank); the
+    identity on one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_us_per_call(ms_per_step: float, calls_per_rank: int, world: int) -> float:
+    """Whole-job time per verify call: every rank runs calls_per_rank calls in
+    a step (weak scaling), the step lasts as long as the slowest rank."""
+    return ms_per_step * 1e3 / (calls_per_rank * world)
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -488,12 +506,9 @@ def run_gpu(args):
             g_step.replay()
         ev1.record(stream)
     torch.cuda.synchronize()
-    ms_total = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), dev)
     if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-        ms_total = float(t.item())
     ms_per_step = ms_total / args.steps
 
     # dominant kernel alone (same grid, partials out): per-launch duration
@@ -558,16 +573,12 @@ def run_gpu(args):
         e2e_step()
     e7.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e6.elapsed_time(e7) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e6.elapsed_time(e7) / e2e_steps, dev)
 
     flops, kv_bytes = case_flops_bytes(c0)
     peaks = load_peaks()
     n_calls = len(prob.params)
-    us_per_call = ms_per_step * 1e3 / (n_calls * world)
+    us_per_call = job_us_per_call(ms_per_step, n_calls, world)
     tc_tflops = flops / (tc_us * 1e-6) / 1e12
     kname, ksrc = TC_KERNEL.get(args.impl_code, TC_KERNEL[2])
     traffic = load_traffic(kname, ksrc) if args.workload == "kimi" else None
