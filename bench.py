@@ -112,7 +112,8 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"], source="fallback")
 
 
-TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 3: ("verify_tc_kernel", "verify_tc.cu")}
+TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 3: ("verify_tc_kernel", "verify_tc.cu"),
+             4: ("verify_tc2_kernel", "verify_tc2.cu")}
 
 
 def kernel_source_hash(src="verify_tc2.cu"):
@@ -314,7 +315,10 @@ class Problems:
             tp = kdv.make_params(**common, num_splits=S, return_partials=1, o=None, lse=None,
                                  o_part=o_part, lse_part=lse_part, workspace=None,
                                  workspace_bytes=0)
-            self.keep += [o_part, lse_part, plen]
+            tbytes = kdv.kdv_verify_attn_workspace(tp)       # staged paged rows, if any
+            tws = torch.empty(max(16, tbytes), dtype=torch.uint8, device=dev)
+            tp.workspace, tp.workspace_bytes = tws.data_ptr(), tbytes
+            self.keep += [o_part, lse_part, plen, tws]
             self.q.append(q); self.kv.append(kv); self.o.append(o); self.lse.append(lse)
             self.ws.append(ws); self.params.append(p); self.tc_params.append(tp)
             self.page_table.append(pt); self.kv_off.append(kv_off); self.tree_off.append(tree_off)
@@ -657,15 +661,16 @@ def main():
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT)
     ap.add_argument("--impl", choices=["kdv", "reference"], default="kdv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["tc2", "tc1"], default="tc2",
-                    help="tensor-core kernel: 2-SM MMAs (default) or 1-SM MMAs")
+    ap.add_argument("--kernel", choices=["tc2", "tc1", "tc2s"], default="tc2",
+                    help="tensor-core kernel: 2-SM MMAs (default), 1-SM MMAs, or 2-SM over a staged "
+                         "contiguous copy of a paged pool")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kimi",
                     help="kimi (default, the headline): " + WORKLOADS["kimi"] + "; sweep: "
                          + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
                          + "; paged: " + WORKLOADS["paged"])
     ap.add_argument("--sweep-L", type=int, choices=SWEEP_L, default=5553)
     args = ap.parse_args()
-    args.impl_code = 2 if args.kernel == "tc2" else 3
+    args.impl_code = {"tc2": 2, "tc1": 3, "tc2s": 4}[args.kernel]
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)

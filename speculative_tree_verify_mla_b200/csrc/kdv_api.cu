@@ -8,6 +8,12 @@
 
 #include "kdv_internal.cuh"
 
+namespace kdv {
+// stage_kv.cu: copy the paged rows of every request to contiguous staged rows
+cudaError_t launch_stage_kv(const VerifyArgs& a, const VerifyPlan& p, int32_t row_bytes, void* staged,
+                            int32_t* staged_off, cudaStream_t stream);
+}  // namespace kdv
+
 using namespace kdv;
 
 namespace {
@@ -28,7 +34,9 @@ bool tc_shape_ok(const kdv_verify_params* p) {
   return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64;
 }
 
-bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_1SM; }
+bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_1SM || impl == KDV_IMPL_TC_STAGED; }
+// the 2-SM kernel, reading the pool directly or a staged copy
+bool is_tc2(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED; }
 
 int resolve_impl(const kdv_verify_params* p) {
   if (p->impl == KDV_IMPL_SIMT || is_tc(p->impl)) return p->impl;
@@ -42,7 +50,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->batch > KDV_MAX_BATCH) return KDV_ERR_UNSUPPORTED;
   if (p->num_heads < 1) return KDV_ERR_INVALID_ARG;
   if (p->dtype != KDV_BF16 && p->dtype != KDV_F32) return KDV_ERR_INVALID_ARG;
-  if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC_1SM) return KDV_ERR_INVALID_ARG;
+  if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC_STAGED) return KDV_ERR_INVALID_ARG;
   if (p->d_latent < 1 || p->d_rope < 0) return KDV_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return KDV_ERR_INVALID_ARG;
   if (p->h_prefix_len == nullptr || p->h_tree_T == nullptr) return KDV_ERR_INVALID_ARG;
@@ -88,11 +96,19 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
   return KDV_OK;
 }
 
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// KDV_IMPL_TC_STAGED with a page table: the pool rows are first copied to a
+// contiguous staged region of the workspace.
+bool staged_paged(const kdv_verify_params* p, int impl) {
+  return impl == KDV_IMPL_TC_STAGED && p->page_table != nullptr;
+}
+
 // Build the grid / split plan. Fills *ws_bytes with the workspace needed.
 kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, size_t* ws_bytes) {
   std::memset(plan, 0, sizeof(*plan));
   const int B = p->batch, H = p->num_heads;
-  const int rows_per_tile = impl == KDV_IMPL_TC ? TC2_ROWS : impl == KDV_IMPL_TC_1SM ? TC_ROWS : SIMT_ROWS;
+  const int rows_per_tile = is_tc2(impl) ? TC2_ROWS : impl == KDV_IMPL_TC_1SM ? TC_ROWS : SIMT_ROWS;
   plan->B = B;
   plan->H = H;
   plan->rows_per_tile = rows_per_tile;
@@ -116,7 +132,7 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   // a GPC, so one wave is what the occupancy query reports (fallback: the SM
   // count divided by the cluster size). SIMT: 8-warp CTAs, several per SM.
   double target_items = 4.0 * sms;
-  if (impl == KDV_IMPL_TC) {
+  if (is_tc2(impl)) {
     const int n = tc2_max_active_clusters();
     target_items = n > 0 ? n : sms / 4;
   } else if (impl == KDV_IMPL_TC_1SM) {
@@ -201,6 +217,14 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
     const size_t o_bytes = (size_t)parts * p->d_latent * sizeof(float);
     const size_t o_al = (o_bytes + 255) & ~(size_t)255;
     *ws_bytes = o_al + (size_t)parts * sizeof(float);
+  }
+  if (staged_paged(p, impl)) {
+    // after the merge region: staged row offsets [B+1], then the staged rows
+    size_t n_keys = 0;
+    for (int b = 0; b < B; ++b) n_keys += (size_t)plan->L[b] + plan->T[b];
+    if (n_keys > (size_t)INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
+    *ws_bytes = align256(*ws_bytes) + align256((size_t)(B + 1) * sizeof(int32_t)) +
+                n_keys * (size_t)(p->d_latent + p->d_rope) * 2;
   }
   return KDV_OK;
 }
@@ -307,7 +331,26 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.lse = ws_l;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = impl == KDV_IMPL_TC       ? launch_verify_tc2(a, plan, s)
+  if (staged_paged(p, impl)) {
+    size_t merge_bytes = 0;
+    if (plan.out_mode == OUT_WORKSPACE) {
+      const size_t parts = (size_t)plan.part_base[plan.B - 1] +
+                           (size_t)plan.S[plan.B - 1] * plan.T[plan.B - 1] * plan.H;
+      merge_bytes = align256(parts * p->d_latent * sizeof(float)) + parts * sizeof(float);
+    }
+    char* region = static_cast<char*>(p->workspace) + align256(merge_bytes);
+    int32_t* staged_off = reinterpret_cast<int32_t*>(region);
+    void* staged = region + align256((size_t)(plan.B + 1) * sizeof(int32_t));
+    int64_t n_keys = 0;
+    for (int b = 0; b < plan.B; ++b) n_keys += (int64_t)plan.L[b] + plan.T[b];
+    cudaError_t e0 = launch_stage_kv(a, plan, (p->d_latent + p->d_rope) * 2, staged, staged_off, s);
+    if (e0 != cudaSuccess) return KDV_ERR_CUDA;
+    a.kv = staged;
+    a.num_slots = n_keys;
+    a.page_table = nullptr;
+    a.kv_off = staged_off;
+  }
+  cudaError_t e = is_tc2(impl)              ? launch_verify_tc2(a, plan, s)
                   : impl == KDV_IMPL_TC_1SM ? launch_verify_tc(a, plan, s)
                                             : launch_verify_simt(a, plan, p->dtype, s);
   if (e != cudaSuccess) return KDV_ERR_CUDA;

@@ -37,6 +37,7 @@ KDV_IMPL_AUTO = 0
 KDV_IMPL_SIMT = 1
 KDV_IMPL_TC = 2
 KDV_IMPL_TC_1SM = 3
+KDV_IMPL_TC_STAGED = 4
 KDV_MAX_TREE = 64
 KDV_MAX_BATCH = 128
 

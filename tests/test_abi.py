@@ -217,3 +217,18 @@ def test_tree_build_validation(lib):
     assert f(parent=None) == kdv.KDV_ERR_INVALID_ARG
     assert f(cand_logp=None) == kdv.KDV_ERR_INVALID_ARG
     assert lib.kdv_tree_build(None, None) == kdv.KDV_ERR_INVALID_ARG
+
+
+def test_staged_workspace_size(lib):
+    # forced single split (no merge region): staged offsets [B+1] then the rows
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC_STAGED,
+                page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
+    assert kdv.kdv_verify_attn_workspace(p) == 256 + 103 * 576 * 2
+    # the gather path needs none
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
+                page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
+    assert kdv.kdv_verify_attn_workspace(p) == 0
+    # impl codes past the last one are rejected
+    n = ctypes.c_size_t(0)
+    assert lib.kdv_verify_attn_workspace(ctypes.byref(_params(impl=5)), ctypes.byref(n)) == \
+        kdv.KDV_ERR_INVALID_ARG

@@ -149,3 +149,38 @@ def test_tc_1sm_rejects_page_table():
     with pytest.raises(kdv.KdvError) as e:
         kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_1SM).run()
     assert e.value.status == kdv.KDV_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# Paged KV through a staged contiguous copy (KDV_IMPL_TC_STAGED).
+
+def test_tc_staged_equals_gather_bit_for_bit():
+    """Staging the rows in logical order and reading them with tiled boxes
+    gives exactly what the four-row gathers give."""
+    parents = [datagen.random_tree(T, np.random.default_rng(T + 7)) for T in (13, 16, 9)]
+    case = datagen.make_case("st", **datagen.KIMI, prefix_len=[2100, 333, 4097], parents=parents,
+                             seed=41, paged=True)
+    for splits in (0, 1, 3):
+        og, lg = _run(case, kdv.KDV_IMPL_TC, splits=splits)
+        os_, ls_ = _run(case, kdv.KDV_IMPL_TC_STAGED, splits=splits)
+        np.testing.assert_array_equal(og, os_)
+        np.testing.assert_array_equal(lg, ls_)
+    o_ref, lse_ref = oracle.verify_case(case)
+    assert_parity(os_, ls_, o_ref, lse_ref)
+
+
+def test_tc_staged_bad_slot_reported():
+    case = datagen.make_case("sb", **datagen.KIMI, prefix_len=[300], parents=[datagen.chain_tree(5)],
+                             seed=3, paged=True)
+    case.page_table = case.page_table.copy()
+    case.page_table[40] = -3
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_STAGED, num_splits=0).run()
+    dc.results()
+    assert dc.error_flag() == kdv.KDV_DERR_BAD_SLOT
+
+
+def test_tc_staged_without_page_table_is_tc():
+    case = datagen.kimi_layer_case(L=900, T=13, seed=5)
+    a = _run(case, kdv.KDV_IMPL_TC, splits=0)
+    b = _run(case, kdv.KDV_IMPL_TC_STAGED, splits=0)
+    np.testing.assert_array_equal(a[0], b[0])
