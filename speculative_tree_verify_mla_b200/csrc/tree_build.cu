@@ -10,13 +10,13 @@
 // that order; with log-probabilities <= 0 this is exactly the best-first
 // expansion (take the best frontier node, add its K children).
 //
-// One CTA per request. The frontier (at most 1 + 64 * 8 entries) lives in
-// shared memory; each of the T rounds is a block-wide argmax over it under
+// One warp per request. The frontier (at most 1 + 64 * 8 entries) lives in
+// shared memory; each of the T rounds is a warp-wide argmax over it under
 // that total order (a unique path key breaks every tie, so the result does
-// not depend on the reduction order), then K threads append the winner's
-// children. The path key holds the choices as D base-(K+1) digits, most
-// significant first, 0 past the path's end: numeric order is digit-by-digit
-// order with a prefix first.
+// not depend on the reduction order), then K lanes append the winner's
+// children -- no block barrier anywhere. The path key holds the choices as
+// D base-(K+1) digits, most significant first, 0 past the path's end:
+// numeric order is digit-by-digit order with a prefix first.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -26,7 +26,7 @@
 namespace kdv {
 namespace {
 
-constexpr int BUILD_THREADS = 256;
+constexpr int BUILD_THREADS = 32;     // one warp per request: no block barriers
 constexpr int MAX_D = 16, MAX_K = 8, MAX_NODES = 64;
 constexpr int MAX_FRONTIER = 1 + MAX_NODES * MAX_K;
 
@@ -65,19 +65,16 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
   __shared__ float s_logp[MAX_D * MAX_K];
   __shared__ int32_t s_tok[MAX_D * MAX_K];
   __shared__ unsigned long long s_place[MAX_D + 1];
-  __shared__ float w_score[BUILD_THREADS / 32];
-  __shared__ unsigned long long w_key[BUILD_THREADS / 32];
-  __shared__ int w_idx[BUILD_THREADS / 32];
-  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int b = blockIdx.x, lane = threadIdx.x;
   const int D = a.D, K = a.K;
   const int t0 = a.tree_off[b];
   const int T = a.tree_off[b + 1] - t0;
-  if (T < 1 || T > a.max_T) {                    // uniform over the block
-    if (t == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);
+  if (T < 1 || T > a.max_T) {                    // uniform over the warp
+    if (lane == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);
     return;
   }
   const int64_t cbase = (int64_t)b * D * K;
-  for (int i = t; i < D * K; i += BUILD_THREADS) {
+  for (int i = lane; i < D * K; i += BUILD_THREADS) {
     float lp = a.cand_logp[cbase + i];
     if (isnan(lp)) {
       record_err(a.d_err, KDV_DERR_BAD_SCORE);
@@ -86,7 +83,7 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
     s_logp[i] = lp;
     s_tok[i] = a.cand_token[cbase + i];
   }
-  if (t == 0) {
+  if (lane == 0) {
     // s_place[d] = (K+1)^(D-d): the weight of the digit chosen at depth d
     unsigned long long p = 1;
     for (int d = D; d >= 1; --d) {
@@ -100,20 +97,29 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
     f_token[0] = a.root_token[b];
     f_live[0] = 1;
   }
-  __syncthreads();
-  int n_front = 1;                                 // uniform: every thread tracks it
+  __syncwarp();
+  int n_front = 1;                                 // uniform over the warp
   int n = 0;
   for (; n < T; ++n) {
-    // ---- best live frontier entry
+    // ---- best live frontier entry: each lane scans a stripe, then shuffles
     float bs = 0.f;
     unsigned long long bk = 0ull;
     int bi = -1;
-    for (int i = t; i < n_front; i += BUILD_THREADS)
-      if (f_live[i] && before(f_score[i], f_key[i], i, bs, bk, bi)) {
-        bs = f_score[i];
-        bk = f_key[i];
-        bi = i;
+    // unrolled over the largest stripe so that a lane's loads issue together
+#pragma unroll
+    for (int st = 0; st < (MAX_FRONTIER + BUILD_THREADS - 1) / BUILD_THREADS; ++st) {
+      const int i = lane + st * BUILD_THREADS;
+      if (i < n_front) {
+        const bool live = f_live[i];
+        const float sc = f_score[i];
+        const unsigned long long ky = f_key[i];
+        if (live && before(sc, ky, i, bs, bk, bi)) {
+          bs = sc;
+          bk = ky;
+          bi = i;
+        }
       }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float os = __shfl_xor_sync(0xffffffffu, bs, o);
@@ -125,48 +131,33 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
         bi = oi;
       }
     }
-    if (lane == 0) {
-      w_score[warp] = bs;
-      w_key[warp] = bk;
-      w_idx[warp] = bi;
-    }
-    __syncthreads();
-    bs = w_score[0];
-    bk = w_key[0];
-    bi = w_idx[0];
-    for (int w = 1; w < BUILD_THREADS / 32; ++w)
-      if (before(w_score[w], w_key[w], w_idx[w], bs, bk, bi)) {
-        bs = w_score[w];
-        bk = w_key[w];
-        bi = w_idx[w];
-      }
     if (bi < 0) break;                             // uniform: candidates ran out
     // ---- emit node n, append its children
     const int dep = f_depth[bi];
-    if (t == 0) {
+    if (lane == 0) {
       a.parent[t0 + n] = f_parent[bi];
       a.token[t0 + n] = f_token[bi];
       if (a.depth) a.depth[t0 + n] = dep;
       if (a.score) a.score[t0 + n] = bs;
     }
     const bool kids = dep < D;
-    if (kids && t < K) {
-      const int i = n_front + t;
-      f_score[i] = bs + s_logp[dep * K + t];
-      f_key[i] = bk + (unsigned long long)(t + 1) * s_place[dep + 1];
+    if (kids && lane < K) {
+      const int i = n_front + lane;
+      f_score[i] = bs + s_logp[dep * K + lane];
+      f_key[i] = bk + (unsigned long long)(lane + 1) * s_place[dep + 1];
       f_depth[i] = dep + 1;
       f_parent[i] = n;
-      f_token[i] = s_tok[dep * K + t];
+      f_token[i] = s_tok[dep * K + lane];
       f_live[i] = 1;
     }
-    __syncthreads();                               // every read of the winner done
-    if (t == 0) f_live[bi] = 0;
+    __syncwarp();                                  // every read of the winner done
+    if (lane == 0) f_live[bi] = 0;
     if (kids) n_front += K;
-    __syncthreads();
+    __syncwarp();
   }
   if (n < T) {                                     // budget above the number of paths
-    if (t == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);
-    for (int i = n + t; i < T; i += BUILD_THREADS) {
+    if (lane == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);
+    for (int i = n + lane; i < T; i += BUILD_THREADS) {
       a.parent[t0 + i] = -1;
       a.token[t0 + i] = -1;
       if (a.depth) a.depth[t0 + i] = 0;
