@@ -96,7 +96,9 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 KDV_API const char* kdv_status_string(kdv_status s);
 
-/* Library ABI version (major*100 + minor). */
+/* Library ABI version (major*100 + minor): 110 adds kdv_tree_accept,
+ * kdv_tree_build, kdv_absorb_q / kdv_unabsorb_o and KDV_IMPL_TC_STAGED to
+ * the 100 set (mask build, verify, no-alloc verify, combine). */
 KDV_API int32_t kdv_version(void);
 
 /*

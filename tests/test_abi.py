@@ -38,7 +38,7 @@ def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4):
         assert kdv.status_string(s).startswith("KDV_")
     assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
-    assert kdv.kdv_version() == 100
+    assert kdv.kdv_version() == 110
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
