@@ -316,12 +316,14 @@ KDV_API kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_lat
  * for each of D future positions, K candidate tokens with log-probabilities;
  * a node is a path of candidate choices (one per position, root = the last
  * committed token at depth 0); its score is the fp32 sum of the chosen
- * log-probabilities, added root first; the tree of request b is the first
- * T_b nodes in (score descending, path ascending digit by digit with a prefix
- * first) order, emitted in that order -- parents precede children, so the
- * output feeds kdv_tree_mask_build directly. With log-probabilities <= 0 this
- * equals the best-first expansion. A NaN log-probability is read as -inf and
- * reported (KDV_DERR_BAD_SCORE). A budget above the number of paths is
+ * log-probabilities, added root first; the tree of request b is what a
+ * best-first expansion emits in T_b steps (take the frontier node first in
+ * (score descending, path ascending digit by digit with a prefix first)
+ * order, add its K children), in emission order -- parents precede
+ * children, so the output feeds kdv_tree_mask_build directly. With
+ * log-probabilities <= 0 this is the first T_b nodes of that order. A NaN log-probability is read as -inf and
+ * reported (KDV_DERR_BAD_SCORE); a path score that comes out NaN (+inf and
+ * -inf on one path) is read as -inf, silently. A budget above the number of paths is
  * reported (KDV_DERR_BAD_LENGTH); the missing nodes get parent -1, token -1.
  */
 typedef struct kdv_tree_build_params {

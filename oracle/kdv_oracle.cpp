@@ -393,8 +393,9 @@ void oracle_accept_commit(int32_t L, int32_t T, int32_t len, const int32_t* path
 // With every logp <= 0 a node never outranks its parent, so this is exactly
 // what a best-first expansion (pop the best frontier node, push its K
 // children) emits. Done here as that expansion with a linear frontier scan.
-// A NaN log-probability is read as -inf (a candidate never preferred), which
-// keeps the order total.
+// A NaN log-probability is read as -inf (a candidate never preferred), and so
+// is a NaN path score (+inf plus -inf along one path): both keep the order
+// total.
 
 namespace {
 struct Cand { float score; uint64_t key; int32_t depth, parent, token; bool live; };
@@ -430,7 +431,9 @@ int oracle_tree_build(int32_t T, int32_t D, int32_t K, int32_t root_token, const
       for (int32_t j = 0; j < K; ++j) {
         float lp = cand_logp[(int64_t)c.depth * K + j];
         if (std::isnan(lp)) lp = -std::numeric_limits<float>::infinity();   // never preferred
-        const float s = c.score + lp;
+        float s = c.score + lp;
+        // +inf + -inf: a path with no defined score is never preferred either
+        if (std::isnan(s)) s = -std::numeric_limits<float>::infinity();
         // the path as D base-(K+1) digits, most significant first, 0 past
         // the end: numeric order = digit-by-digit order with a prefix first
         uint64_t place = 1;

@@ -5,30 +5,38 @@
 // grows the draft tree best-first. A block drafter proposes K candidate
 // tokens with log-probabilities for each of D future positions; a node is a
 // path of candidate choices, its score the fp32 sum of the log-probabilities
-// along it (one float add per edge, root first). The tree is the first T
-// nodes in (score descending, candidate path ascending) order, emitted in
-// that order; with log-probabilities <= 0 this is exactly the best-first
-// expansion (take the best frontier node, add its K children).
+// along it (one float add per edge, root first). The tree is what T steps of
+// best-first expansion emit (take the frontier node first in (score
+// descending, candidate path ascending) order, add its K children); with
+// log-probabilities <= 0 that is the first T nodes of that order.
 //
-// One warp per request. The frontier (at most 1 + 64 * 8 entries) lives in
-// shared memory; each of the T rounds is a warp-wide argmax over it under
-// that total order (a unique path key breaks every tie, so the result does
-// not depend on the reduction order), then K lanes append the winner's
-// children -- no block barrier anywhere. The path key holds the choices as
-// D base-(K+1) digits, most significant first, 0 past the path's end:
-// numeric order is digit-by-digit order with a prefix first.
+// One warp per request, no block barrier anywhere. Frontier entry i belongs
+// to lane i % 32, which alone writes and reads its fields in shared memory;
+// every lane keeps the best of its own live entries in registers. A round is
+// then a warp-wide selection of the best lane-best under that total order
+// (redux max over an order-preserving integer image of the score, redux min
+// over the unique path key only when scores tie), after which the winner's
+// lane retires it and rescans its own entries while the K lanes that own the
+// next K frontier slots append the winner's children. The path key holds the
+// choices as D base-(K+1) digits, most significant first, 0 past the path's
+// end: numeric order is digit-by-digit order with a prefix first. A child's
+// score that comes out NaN (+inf plus -inf) is read as -inf, like a NaN
+// log-probability: a path with no defined score is never preferred.
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdint>
 
 #include "kdv.h"
 
 namespace kdv {
 namespace {
 
-constexpr int BUILD_THREADS = 32;     // one warp per request: no block barriers
+constexpr int BUILD_THREADS = 32;     // one warp per request
 constexpr int MAX_D = 16, MAX_K = 8, MAX_NODES = 64;
 constexpr int MAX_FRONTIER = 1 + MAX_NODES * MAX_K;
+constexpr int NSTRIPE = (MAX_FRONTIER + BUILD_THREADS - 1) / BUILD_THREADS;
+constexpr unsigned FULL = 0xffffffffu;
 
 struct BuildArgs {
   int32_t max_T, D, K;
@@ -47,21 +55,26 @@ __device__ __forceinline__ void record_err(int32_t* d_err, int32_t code) {
   if (d_err != nullptr) atomicCAS(d_err, 0, code);
 }
 
-// a ranks before b (score descending, then key ascending); an empty slot
-// (idx < 0) ranks last
-__device__ __forceinline__ bool before(float sa, unsigned long long ka, int ia, float sb, unsigned long long kb,
-                                       int ib) {
-  if (ia < 0) return false;
-  if (ib < 0) return true;
-  if (sa != sb) return sa > sb;
-  return ka < kb;
+// Order-preserving image of a non-NaN score in [1, 2^32): x < y <=> img(x) <
+// img(y), +0 and -0 equal. 0 stands for "no live entry".
+__device__ __forceinline__ uint32_t score_img(float s) {
+  const uint32_t u = __float_as_uint(s == 0.f ? 0.f : s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float score_of(uint32_t img) {
+  return __uint_as_float((img & 0x80000000u) ? (img & 0x7fffffffu) : ~img);
+}
+
+// (img, key) a ranks before b: score descending, then path key ascending
+__device__ __forceinline__ bool before(uint32_t ia, unsigned long long ka, uint32_t ib, unsigned long long kb) {
+  return ia > ib || (ia == ib && ka < kb);
 }
 
 __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildArgs a) {
-  __shared__ float f_score[MAX_FRONTIER];
-  __shared__ unsigned long long f_key[MAX_FRONTIER];
-  __shared__ int32_t f_depth[MAX_FRONTIER], f_parent[MAX_FRONTIER], f_token[MAX_FRONTIER];
-  __shared__ unsigned char f_live[MAX_FRONTIER];
+  // frontier entries; entry i is touched by lane i % 32 only
+  __shared__ uint32_t e_img[MAX_FRONTIER];
+  __shared__ unsigned long long e_key[MAX_FRONTIER];
+  __shared__ int32_t e_depth[MAX_FRONTIER], e_parent[MAX_FRONTIER], e_token[MAX_FRONTIER];
   __shared__ float s_logp[MAX_D * MAX_K];
   __shared__ int32_t s_tok[MAX_D * MAX_K];
   __shared__ unsigned long long s_place[MAX_D + 1];
@@ -73,87 +86,129 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
     if (lane == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);
     return;
   }
+  // ---- candidates into shared memory: every load issued before any use
   const int64_t cbase = (int64_t)b * D * K;
-  for (int i = lane; i < D * K; i += BUILD_THREADS) {
-    float lp = a.cand_logp[cbase + i];
-    if (isnan(lp)) {
-      record_err(a.d_err, KDV_DERR_BAD_SCORE);
-      lp = -INFINITY;                              // a candidate never preferred
+  constexpr int PER_LANE = MAX_D * MAX_K / BUILD_THREADS;
+  float lp[PER_LANE];
+  int32_t tk[PER_LANE];
+#pragma unroll
+  for (int r = 0; r < PER_LANE; ++r) {
+    const int i = lane + r * BUILD_THREADS;
+    if (i < D * K) {
+      lp[r] = a.cand_logp[cbase + i];
+      tk[r] = a.cand_token[cbase + i];
     }
-    s_logp[i] = lp;
-    s_tok[i] = a.cand_token[cbase + i];
   }
-  if (lane == 0) {
-    // s_place[d] = (K+1)^(D-d): the weight of the digit chosen at depth d
+#pragma unroll
+  for (int r = 0; r < PER_LANE; ++r) {
+    const int i = lane + r * BUILD_THREADS;
+    if (i < D * K) {
+      if (isnan(lp[r])) {
+        record_err(a.d_err, KDV_DERR_BAD_SCORE);
+        lp[r] = -INFINITY;                           // a candidate never preferred
+      }
+      s_logp[i] = lp[r];
+      s_tok[i] = tk[r];
+    }
+  }
+  if (lane >= 1 && lane <= D) {                    // s_place[d] = (K+1)^(D-d)
     unsigned long long p = 1;
-    for (int d = D; d >= 1; --d) {
-      s_place[d] = p;
-      p *= (unsigned long long)(K + 1);
-    }
-    f_score[0] = 0.f;
-    f_key[0] = 0ull;
-    f_depth[0] = 0;
-    f_parent[0] = -1;
-    f_token[0] = a.root_token[b];
-    f_live[0] = 1;
+    for (int e = lane; e < D; ++e) p *= (unsigned long long)(K + 1);
+    s_place[lane] = p;
   }
-  __syncwarp();
+  // ---- the root: entry 0, lane 0
+  uint32_t lb_img = 0;                             // this lane's best live entry
+  unsigned long long lb_key = 0ull;
+  int lb_dep = 0, lb_idx = -1;
+  if (lane == 0) {
+    e_img[0] = score_img(0.f);
+    e_key[0] = 0ull;
+    e_depth[0] = 0;
+    e_parent[0] = -1;
+    e_token[0] = a.root_token[b];
+    lb_img = score_img(0.f);
+    lb_idx = 0;
+  }
+  __syncwarp();                                    // candidates visible to every lane
   int n_front = 1;                                 // uniform over the warp
   int n = 0;
   for (; n < T; ++n) {
-    // ---- best live frontier entry: each lane scans a stripe, then shuffles
-    float bs = 0.f;
-    unsigned long long bk = 0ull;
-    int bi = -1;
-    // unrolled over the largest stripe so that a lane's loads issue together
-#pragma unroll
-    for (int st = 0; st < (MAX_FRONTIER + BUILD_THREADS - 1) / BUILD_THREADS; ++st) {
-      const int i = lane + st * BUILD_THREADS;
-      if (i < n_front) {
-        const bool live = f_live[i];
-        const float sc = f_score[i];
-        const unsigned long long ky = f_key[i];
-        if (live && before(sc, ky, i, bs, bk, bi)) {
-          bs = sc;
-          bk = ky;
-          bi = i;
-        }
-      }
+    // ---- the best live entry of the warp
+    const uint32_t m = __reduce_max_sync(FULL, lb_img);
+    if (m == 0u) break;                            // uniform: candidates ran out
+    uint32_t win = __ballot_sync(FULL, lb_img == m);
+    if (__popc(win) > 1) {                         // uniform: tied scores, unique keys decide
+      const bool t = (win >> lane) & 1u;
+      const uint32_t khi = t ? (uint32_t)(lb_key >> 32) : 0xffffffffu;
+      const uint32_t mh = __reduce_min_sync(FULL, khi);
+      const bool t2 = t && khi == mh;
+      const uint32_t klo = t2 ? (uint32_t)lb_key : 0xffffffffu;
+      const uint32_t ml = __reduce_min_sync(FULL, klo);
+      win = __ballot_sync(FULL, t2 && klo == ml);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-      const unsigned long long ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (before(os, ok, oi, bs, bk, bi)) {
-        bs = os;
-        bk = ok;
-        bi = oi;
-      }
-    }
-    if (bi < 0) break;                             // uniform: candidates ran out
-    // ---- emit node n, append its children
-    const int dep = f_depth[bi];
-    if (lane == 0) {
-      a.parent[t0 + n] = f_parent[bi];
-      a.token[t0 + n] = f_token[bi];
+    const int owner = __ffs(win) - 1;
+    const unsigned long long bk = __shfl_sync(FULL, lb_key, owner);
+    const int bi = __shfl_sync(FULL, lb_idx, owner);
+    const int dep = __shfl_sync(FULL, lb_dep, owner);
+    const float bs = score_of(m);
+    // ---- the winner's lane emits node n, retires it and rescans its entries
+    if (lane == owner) {
+      a.parent[t0 + n] = e_parent[bi];
+      a.token[t0 + n] = e_token[bi];
       if (a.depth) a.depth[t0 + n] = dep;
       if (a.score) a.score[t0 + n] = bs;
+      e_img[bi] = 0u;
+      uint32_t c_img[NSTRIPE];
+      unsigned long long c_key[NSTRIPE];
+      int c_st[NSTRIPE];
+#pragma unroll
+      for (int st = 0; st < NSTRIPE; ++st) {
+        const int i = lane + st * BUILD_THREADS;
+        const bool have = i < n_front;
+        c_img[st] = have ? e_img[i] : 0u;
+        c_key[st] = have ? e_key[i] : 0ull;
+        c_st[st] = st;
+      }
+      // pairwise tournament: 5 levels instead of a 16-long chain
+#pragma unroll
+      for (int w = 1; w < NSTRIPE; w *= 2) {
+#pragma unroll
+        for (int st = 0; st + w < NSTRIPE; st += 2 * w) {
+          if (before(c_img[st + w], c_key[st + w], c_img[st], c_key[st])) {
+            c_img[st] = c_img[st + w];
+            c_key[st] = c_key[st + w];
+            c_st[st] = c_st[st + w];
+          }
+        }
+      }
+      lb_img = c_img[0];
+      lb_key = c_key[0];
+      lb_idx = lane + c_st[0] * BUILD_THREADS;
+      lb_dep = lb_img != 0u ? e_depth[lb_idx] : 0;
     }
-    const bool kids = dep < D;
-    if (kids && lane < K) {
-      const int i = n_front + lane;
-      f_score[i] = bs + s_logp[dep * K + lane];
-      f_key[i] = bk + (unsigned long long)(lane + 1) * s_place[dep + 1];
-      f_depth[i] = dep + 1;
-      f_parent[i] = n;
-      f_token[i] = s_tok[dep * K + lane];
-      f_live[i] = 1;
+    // ---- the lanes owning slots n_front .. n_front+K-1 append the children
+    if (dep < D) {                                 // uniform
+      const int j = (lane - n_front) & (BUILD_THREADS - 1);
+      if (j < K) {
+        const int i = n_front + j;                 // i % 32 == lane
+        float sc = bs + s_logp[dep * K + j];
+        if (isnan(sc)) sc = -INFINITY;             // +inf + -inf: no defined score
+        const uint32_t img = score_img(sc);
+        const unsigned long long ky = bk + (unsigned long long)(j + 1) * s_place[dep + 1];
+        e_img[i] = img;
+        e_key[i] = ky;
+        e_depth[i] = dep + 1;
+        e_parent[i] = n;
+        e_token[i] = s_tok[dep * K + j];
+        if (lb_img == 0u || before(img, ky, lb_img, lb_key)) {
+          lb_img = img;
+          lb_key = ky;
+          lb_idx = i;
+          lb_dep = dep + 1;
+        }
+      }
+      n_front += K;
     }
-    __syncwarp();                                  // every read of the winner done
-    if (lane == 0) f_live[bi] = 0;
-    if (kids) n_front += K;
-    __syncwarp();
   }
   if (n < T) {                                     // budget above the number of paths
     if (lane == 0) record_err(a.d_err, KDV_DERR_BAD_LENGTH);

@@ -74,3 +74,28 @@ def test_build_nan_logprob_reported_and_read_as_minus_inf():
     case.cand_logp = case.cand_logp.copy()
     case.cand_logp[0, 1, 2] = np.nan
     _check(case, expect_err=kdv.KDV_DERR_BAD_SCORE)
+
+
+def test_build_nan_path_score_silent_minus_inf():
+    """+inf then -inf on one path: the NaN sum ranks as -inf, not reported."""
+    case = datagen.make_build_case([40, 15], D=3, K=2, seed=6)
+    case.cand_logp = case.cand_logp.copy()
+    case.cand_logp[0, 0, 0] = np.inf
+    case.cand_logp[0, 1, 0] = -np.inf
+    case.cand_logp[1, 2, 1] = np.inf
+    _check(case, expect_err=kdv.KDV_DERR_BAD_LENGTH)   # 15 paths < 40
+
+
+@pytest.mark.parametrize("value", [0.0, -np.inf, -1.0])
+def test_build_all_scores_tied_keys_decide(value):
+    """Every candidate with one log-probability: depth-16, K = 8 keys exceed
+    32 bits, so the path-key tie-break runs on both halves of the key."""
+    case = datagen.make_build_case([64, 64, 33, 5], D=16, K=8, seed=7)
+    case.cand_logp = np.full_like(case.cand_logp, value)
+    _check(case)
+
+
+def test_build_full_batch():
+    rng = np.random.default_rng(8)
+    budgets = [int(x) for x in rng.integers(1, 65, size=kdv.KDV_MAX_BATCH)]
+    _check(datagen.make_build_case(budgets, seed=9))

@@ -109,3 +109,32 @@ def test_build_nan_logprob_reads_as_minus_inf():
     a = oracle.tree_build(30, 5, cand_token, with_nan)
     b = _brute_force(30, 5, cand_token, with_inf)
     assert list(a[0]) == b[0] and list(a[1]) == b[1]
+
+
+def test_build_nan_path_score_reads_as_minus_inf():
+    """+inf at one position and -inf at the next make the path's fp32 sum NaN;
+    that path ranks like a -inf one. With a +inf log-probability a child can
+    outrank its parent, so the reference here is a plain best-first expansion
+    (frontier as a Python list, best = min of (-score, path)) with NaN sums
+    replaced by -inf."""
+    cand_token = np.array([[10, 11], [20, 21], [30, 31]], dtype=np.int32)
+    cand_logp = np.array([[np.inf, -0.5], [-np.inf, -0.25], [-1.0, -2.0]], dtype=np.float32)
+    got = oracle.tree_build(15, 3, cand_token, cand_logp)
+
+    D, K = cand_token.shape
+    frontier = [((), np.float32(0.0), -1)]
+    out = []
+    with np.errstate(invalid="ignore"):
+        while frontier and len(out) < 15:
+            best = min(range(len(frontier)), key=lambda i: (-float(frontier[i][1]), frontier[i][0]))
+            path, sc, par = frontier.pop(best)
+            out.append((path, sc, par))
+            if len(path) < D:
+                for j in range(K):
+                    s = np.float32(sc + cand_logp[len(path), j])
+                    frontier.append((path + (j,), np.float32(-np.inf) if np.isnan(s) else s, len(out) - 1))
+    assert list(got[0]) == [par for _, _, par in out]
+    assert list(got[2]) == [len(p) for p, _, _ in out]
+    assert [float(x) for x in got[3]] == [float(s) for _, s, _ in out]
+    # the paths under (0, 0) are the NaN ones
+    assert any(p[:2] == (0, 0) and np.isneginf(s) for p, s, _ in out)
