@@ -8,13 +8,20 @@
 // Rows are node-major (row = t*H + h), so head h owns rows h, H+h, 2H+h, ...
 // Both read every weight once per call (2 x 8.4 MB in bf16 for the Kimi shape)
 // and do ~2*T flops per weight, so they are HBM-bound; the arithmetic is
-// fp32 on CUDA cores. Both kernels stage a head's input rows in shared
-// memory and issue each thread's weight loads before any arithmetic, so the
-// weights stream in one memory round trip.
+// fp32 on CUDA cores. The main kernels (bf16 weights whose rows are a
+// multiple of 16 bytes) bring a CTA's whole weight tile into shared memory
+// with one round of TMA copies and keep many warps busy on it: each thread
+// holds a small block of outputs (two weight rows x four nodes, or four
+// columns x four nodes) so that every shared-memory read feeds several packed
+// fp32 FMAs (two correctly rounded fp32 FMAs per instruction). The general
+// kernels below them (fp32 weights, other alignments) stage a head's input
+// rows and issue each thread's weight loads before any arithmetic.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kdv.h"
+#include "sm100_ptx.cuh"
 
 namespace kdv {
 namespace {
@@ -235,6 +242,289 @@ unabsorb_o_kernel(int32_t rows_per_head, int32_t H, int32_t D_c, int32_t D_v, co
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// TMA-staged kernels (bf16 weights)
+// ---------------------------------------------------------------------------
+constexpr int P_THREADS = 256;
+constexpr int PA_ROWS = 128;         // absorb: weight rows (d) per CTA
+constexpr int PA_TB = 16;            // absorb: nodes per pass (4 groups x 4)
+constexpr int PU_V = 32;             // unabsorb: output columns per CTA
+constexpr int PU_TB = 16;            // unabsorb: nodes per pass (4 groups x 4)
+constexpr int PU_DG = 8;             // unabsorb: d interleave (d = g + 8 j)
+constexpr int PU_MAX_DC = 512;
+constexpr unsigned long long WAIT_NS = 2000000000ull;   // a TMA that has not landed in 2 s never will
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase 0 of `bar`, for at most WAIT_NS; false if it never completed.
+__device__ __forceinline__ bool wait_landed(uint32_t bar) {
+  if (ptx::mbar_try_wait(bar, 0)) return true;
+  const unsigned long long t0 = gtimer();
+  while (!ptx::mbar_try_wait(bar, 0))
+    if (gtimer() - t0 > WAIT_NS) return false;
+  return true;
+}
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) { return make_float2(bf16_lo(w), bf16_hi(w)); }
+
+// Stage rows [r0, r0+nr) of head h into shared memory as fp32 (DUP: as
+// (x, x) pairs), 8 elements per 16- or 32-byte unit, every load of a thread
+// issued before its first store. Needs n % 8 == 0, a 16-byte aligned base
+// and a row stride that is a multiple of 8 elements.
+template <bool DUP>
+__device__ __forceinline__ void stage_rows_vec(void* dst, const void* src, int dtype, int64_t stride, int r0, int nr,
+                                               int H, int h, int n) {
+  constexpr int U = 4;
+  const int units = n / 8, total = nr * units;
+  for (int base = threadIdx.x; base < total; base += P_THREADS * U) {
+    float v[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * P_THREADS;
+      if (i < total) {
+        const int r = i / units, k8 = (i - r * units) * 8;
+        const int64_t e = (int64_t)((r0 + r) * H + h) * stride + k8;
+        if (dtype == KDV_BF16) {
+          const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + e);
+          v[u][0] = bf16_lo(w.x); v[u][1] = bf16_hi(w.x); v[u][2] = bf16_lo(w.y); v[u][3] = bf16_hi(w.y);
+          v[u][4] = bf16_lo(w.z); v[u][5] = bf16_hi(w.z); v[u][6] = bf16_lo(w.w); v[u][7] = bf16_hi(w.w);
+        } else {
+          const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + e);
+          const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + e + 4);
+          v[u][0] = a.x; v[u][1] = a.y; v[u][2] = a.z; v[u][3] = a.w;
+          v[u][4] = b.x; v[u][5] = b.y; v[u][6] = b.z; v[u][7] = b.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * P_THREADS;
+      if (i < total) {
+        const int r = i / units, k8 = (i - r * units) * 8;
+        if (DUP) {
+          float4* d4 = reinterpret_cast<float4*>(static_cast<float2*>(dst) + r * n + k8);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) d4[j] = make_float4(v[u][2 * j], v[u][2 * j], v[u][2 * j + 1], v[u][2 * j + 1]);
+        } else {
+          float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + r * n + k8);
+          d4[0] = make_float4(v[u][0], v[u][1], v[u][2], v[u][3]);
+          d4[1] = make_float4(v[u][4], v[u][5], v[u][6], v[u][7]);
+        }
+      }
+    }
+  }
+}
+
+// q_lat[row][d] = sum_k W_UK[h][d][k] q_nope[row][k]. CTA = (128 rows d of
+// head h); its W_UK tile arrives as ceil(D_n/64) TMA boxes of [128 rows][64 k]
+// with the 128-byte swizzle (16-byte chunk c of row r sits at chunk c ^ (r%8)),
+// so the 32 rows a warp reads at one k land in distinct banks. Thread
+// (rp = tid % 64, tg = tid / 64) owns rows rp and rp + 64 and nodes tg,
+// tg+4, tg+8, tg+12 of each 16-node pass; a warp shares its nodes, so the
+// node reads are broadcasts. k runs in pairs: the even and odd k of a row
+// accumulate in the two halves of a float2 and are added at the end.
+__global__ void __launch_bounds__(P_THREADS)
+absorb_q_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per_head, int32_t H, int32_t D_c,
+                    int32_t D_n, const void* __restrict__ q_nope, int64_t q_stride, int q_dtype, int q_vec,
+                    void* __restrict__ q_lat, int64_t o_stride, int o_dtype) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) unsigned long long bar;
+  unsigned char* s_w = align1024(smem_raw);
+  const int nbox = (D_n + 63) / 64;
+  float* s_q = reinterpret_cast<float*>(s_w + nbox * 16384);      // [PA_TB][D_n]
+  const int h = blockIdx.y, d0 = blockIdx.x * PA_ROWS;
+  const uint32_t b = ptx::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(b, 1);
+    ptx::fence_mbar_init();
+    ptx::mbar_arrive_expect_tx(b, (uint32_t)nbox * 16384u);
+    for (int i = 0; i < nbox; ++i) ptx::tma_load_2d(ptx::smem_u32(s_w + i * 16384), &tmap_w, b, i * 64, h * D_c + d0);
+  }
+  const int rp = threadIdx.x & 63, tg = threadIdx.x >> 6;
+  const int ra = rp, rb = rp + 64;
+  const int da = d0 + ra, db = d0 + rb;
+  bool landed = false, ok = true;
+  for (int tb0 = 0; tb0 < rows_per_head; tb0 += PA_TB) {
+    const int nr = min(PA_TB, rows_per_head - tb0);
+    __syncthreads();                                 // barrier init seen; s_q free
+    if (q_vec) stage_rows_vec<false>(s_q, q_nope, q_dtype, q_stride, tb0, nr, H, h, D_n);
+    else stage_rows(s_q, q_nope, q_dtype, q_stride, tb0, nr, H, h, D_n, P_THREADS);
+    __syncthreads();
+    if (!landed) {
+      ok = wait_landed(b);
+      landed = true;
+    }
+    float2 acc[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+    const int nchunk = D_n / 8;
+    for (int c = 0; c < nchunk; ++c) {
+      const unsigned char* box = s_w + (c >> 3) * 16384;
+      const int cc = c & 7;
+      const uint4 wa = *reinterpret_cast<const uint4*>(box + ra * 128 + ((cc ^ (ra & 7)) << 4));
+      const uint4 wb = *reinterpret_cast<const uint4*>(box + rb * 128 + ((cc ^ (rb & 7)) << 4));
+      const float2 fa[4] = {bf16x2_to_float2(wa.x), bf16x2_to_float2(wa.y), bf16x2_to_float2(wa.z),
+                            bf16x2_to_float2(wa.w)};
+      const float2 fb[4] = {bf16x2_to_float2(wb.x), bf16x2_to_float2(wb.y), bf16x2_to_float2(wb.z),
+                            bf16x2_to_float2(wb.w)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = tg + 4 * i;
+        if (t < nr) {                                // uniform over the warp
+          const float4 q0 = *reinterpret_cast<const float4*>(s_q + t * D_n + 8 * c);
+          const float4 q1 = *reinterpret_cast<const float4*>(s_q + t * D_n + 8 * c + 4);
+          const float2 p[4] = {make_float2(q0.x, q0.y), make_float2(q0.z, q0.w), make_float2(q1.x, q1.y),
+                               make_float2(q1.z, q1.w)};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[i][0] = __ffma2_rn(fa[j], p[j], acc[i][0]);
+            acc[i][1] = __ffma2_rn(fb[j], p[j], acc[i][1]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tg + 4 * i;
+      if (t < nr) {
+        const int64_t row = (int64_t)(tb0 + t) * H + h;
+        if (da < D_c) st_elem(q_lat, row * o_stride + da, o_dtype, ok ? acc[i][0].x + acc[i][0].y : __int_as_float(0x7fc00000));
+        if (db < D_c) st_elem(q_lat, row * o_stride + db, o_dtype, ok ? acc[i][1].x + acc[i][1].y : __int_as_float(0x7fc00000));
+      }
+    }
+  }
+}
+
+// out[row][v] = sum_d W_UV[h][d][v] o_lat[row][d]. CTA = (32 columns of head
+// h); its W_UV slice [D_c rows][32 v] arrives as TMA boxes of [256 rows][32 v]
+// (64-byte rows, no swizzle). Thread (q = v quad, g = d phase, tg = node
+// group) accumulates columns 4q..4q+3 for nodes tg, tg+4, tg+8, tg+12 over
+// d = g, g+8, g+16, ...; a warp is 8 quads x 4 consecutive phases, so its
+// weight reads cover 256 contiguous bytes and its node reads 4 words. Node
+// rows are staged duplicated ((o, o) pairs) so one 8-byte read gives the
+// packed-FMA operand. The 8 phases' partial sums are added in shared memory.
+__global__ void __launch_bounds__(P_THREADS)
+unabsorb_o_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per_head, int32_t H, int32_t D_c,
+                      int32_t D_v, const float* __restrict__ o_lat, int64_t i_stride, int o_vec,
+                      void* __restrict__ out, int64_t o_stride, int o_dtype) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) unsigned long long bar;
+  unsigned char* s_w = align1024(smem_raw);                   // [D_c padded to 256][32] bf16
+  const int nbox = (D_c + 255) / 256;
+  float2* s_o = reinterpret_cast<float2*>(s_w + nbox * 256 * PU_V * 2);   // [PU_TB][D_c] (o, o)
+  float* s_part = reinterpret_cast<float*>(s_o);                          // reused: [PU_DG][PU_TB][PU_V]
+  const int h = blockIdx.y, v0 = blockIdx.x * PU_V;
+  const uint32_t b = ptx::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(b, 1);
+    ptx::fence_mbar_init();
+    ptx::mbar_arrive_expect_tx(b, (uint32_t)nbox * 256u * PU_V * 2u);
+    for (int i = 0; i < nbox; ++i)
+      ptx::tma_load_2d(ptx::smem_u32(s_w + i * 256 * PU_V * 2), &tmap_w, b, v0, h * D_c + i * 256);
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int q = lane & 7;                                     // columns 4q .. 4q+3
+  const int g = (lane >> 3) + 4 * (w & 1);                    // d phase 0..7
+  const int tg = w >> 1;                                      // node group 0..3
+  bool landed = false, ok = true;
+  for (int tb0 = 0; tb0 < rows_per_head; tb0 += PU_TB) {
+    const int nr = min(PU_TB, rows_per_head - tb0);
+    __syncthreads();                                          // barrier init seen; s_o / s_part free
+    if (o_vec) {
+      stage_rows_vec<true>(s_o, o_lat, KDV_F32, i_stride, tb0, nr, H, h, D_c);
+    } else {
+      for (int i = threadIdx.x; i < nr * D_c; i += P_THREADS) {
+        const int r = i / D_c, d = i - r * D_c;
+        const float x = o_lat[((int64_t)(tb0 + r) * H + h) * i_stride + d];
+        s_o[r * D_c + d] = make_float2(x, x);
+      }
+    }
+    __syncthreads();
+    if (!landed) {
+      ok = wait_landed(b);
+      landed = true;
+    }
+    float2 acc[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+    for (int d = g; d < D_c; d += PU_DG) {
+      const uint2 wv = *reinterpret_cast<const uint2*>(s_w + d * (PU_V * 2) + q * 8);
+      const float2 f0 = bf16x2_to_float2(wv.x), f1 = bf16x2_to_float2(wv.y);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = tg + 4 * i;
+        if (t < nr) {                                         // uniform over the warp
+          const float2 o2 = s_o[t * D_c + d];
+          acc[i][0] = __ffma2_rn(f0, o2, acc[i][0]);
+          acc[i][1] = __ffma2_rn(f1, o2, acc[i][1]);
+        }
+      }
+    }
+    __syncthreads();                                          // every read of s_o done
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = tg + 4 * i;
+      if (t < nr) {
+        float* dst = s_part + (g * PU_TB + t) * PU_V + 4 * q;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y);
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nr * PU_V; i += P_THREADS) {
+      const int t = i / PU_V, col = i - t * PU_V, v = v0 + col;
+      float sum = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < PU_DG; ++gg) sum += s_part[(gg * PU_TB + t) * PU_V + col];
+      if (v < D_v)
+        st_elem(out, ((int64_t)(tb0 + t) * H + h) * o_stride + v, o_dtype, ok ? sum : __int_as_float(0x7fc00000));
+    }
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 weights [rows][cols] (row pitch = cols) as a 2D tensor map with boxes
+// of [box_rows][box_cols]; false if the driver refuses it.
+bool weight_map(CUtensorMap* m, const void* w, uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows,
+                CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t absorb_tma_smem(int D_n) { return 1024 + (size_t)((D_n + 63) / 64) * 16384 + (size_t)PA_TB * D_n * 4; }
+size_t unabsorb_tma_smem(int D_c) {
+  const size_t part = (size_t)PU_DG * PU_TB * PU_V * 4, o = (size_t)PU_TB * D_c * 8;
+  return 1024 + (size_t)((D_c + 255) / 256) * 256 * PU_V * 2 + (o > part ? o : part);
+}
+
 bool dtype_ok(int d) { return d == KDV_BF16 || d == KDV_F32; }
 
 kdv_status check_common(int32_t rows, int32_t H, int32_t D_in, int32_t D_out, const void* in, int64_t in_stride,
@@ -272,12 +562,25 @@ kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32
     if (cudaFuncSetAttribute(absorb_q_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, RCH * 512 * 4) !=
             cudaSuccess ||
         cudaFuncSetAttribute(absorb_q_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, RCH * 512 * 4) !=
-            cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(absorb_q_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)absorb_tma_smem(512)) != cudaSuccess)
       return KDV_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const dim3 grid((unsigned)num_heads, (unsigned)((d_latent + THREADS - 1) / THREADS));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tmap;
+  if (vec && (int64_t)num_heads * d_latent <= 0x7fffffff &&
+      weight_map(&tmap, w_uk, (uint64_t)num_heads * d_latent, (uint64_t)d_nope, 64, PA_ROWS,
+                 CU_TENSOR_MAP_SWIZZLE_128B)) {
+    const dim3 g2((unsigned)((d_latent + PA_ROWS - 1) / PA_ROWS), (unsigned)num_heads);
+    absorb_q_tma_kernel<<<g2, P_THREADS, absorb_tma_smem(d_nope), s>>>(
+        tmap, rows / num_heads, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_dtype,
+        (reinterpret_cast<uintptr_t>(q_nope) & 15) == 0 && q_nope_stride % 8 == 0 ? 1 : 0, q_lat, q_lat_stride,
+        out_dtype);
+    return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)num_heads, (unsigned)((d_latent + THREADS - 1) / THREADS));
   if (vec)
     absorb_q_kernel<true><<<grid, THREADS, smem, s>>>(rows / num_heads, num_heads, d_latent, d_nope, q_nope,
                                                       q_nope_stride, q_dtype, w_uk, w_dtype, q_lat, q_lat_stride,
@@ -306,12 +609,26 @@ kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int
     if (cudaFuncSetAttribute(unabsorb_o_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
             cudaSuccess ||
         cudaFuncSetAttribute(unabsorb_o_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-            cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(unabsorb_o_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)unabsorb_tma_smem(PU_MAX_DC)) != cudaSuccess)
       return KDV_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const dim3 grid((unsigned)num_heads, (unsigned)((d_v + U_VB - 1) / U_VB));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tmap;
+  if (w_dtype == KDV_BF16 && d_v % 8 == 0 && d_latent <= PU_MAX_DC &&
+      (reinterpret_cast<uintptr_t>(w_uv) & 15) == 0 && (int64_t)num_heads * d_latent <= 0x7fffffff &&
+      weight_map(&tmap, w_uv, (uint64_t)num_heads * d_latent, (uint64_t)d_v, PU_V, 256,
+                 CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    const dim3 g2((unsigned)((d_v + PU_V - 1) / PU_V), (unsigned)num_heads);
+    unabsorb_o_tma_kernel<<<g2, P_THREADS, unabsorb_tma_smem(d_latent), s>>>(
+        tmap, rows / num_heads, num_heads, d_latent, d_v, o_lat, o_lat_stride,
+        (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0 && o_lat_stride % 8 == 0 && d_latent % 8 == 0 ? 1 : 0, out,
+        out_stride, out_dtype);
+    return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+  }
+  const dim3 grid((unsigned)num_heads, (unsigned)((d_v + U_VB - 1) / U_VB));
   if (w_dtype == KDV_BF16)
     unabsorb_o_kernel<true><<<grid, U_THREADS, smem, s>>>(rows / num_heads, num_heads, d_latent, d_v, o_lat,
                                                           o_lat_stride, w_uv, w_dtype, out, out_stride, out_dtype);

@@ -72,6 +72,37 @@ def test_unabsorb_o_kimi(T, out_dt):
         assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-6)
 
 
+def _bf16_exact(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).bfloat16().float().numpy()
+
+
+@pytest.mark.parametrize("H,T,D_c,D_n,D_v,pad", [(3, 5, 200, 72, 40, 0), (2, 17, 136, 8, 8, 0),
+                                                 (1, 33, 512, 512, 96, 0), (2, 3, 100, 16, 24, 3)])
+def test_projections_ragged_shapes_bf16_weights(H, T, D_c, D_n, D_v, pad):
+    """bf16 weights with shapes that leave every tile ragged: weight rows not
+    a multiple of the 128-row tile, k not a multiple of the 64-wide box, d not
+    a multiple of the 8-way phase split, columns not a multiple of 32, and node
+    counts across several 16-node passes; pad > 0 gives the input rows a
+    stride that is not a multiple of 8 elements (element-wise staging)."""
+    rng = np.random.default_rng(H * 1000 + T)
+    rows = H * T
+    q_nope = _bf16_exact(rng.standard_normal((rows, D_n)))
+    w_uk = _bf16_exact(rng.standard_normal((H, D_c, D_n)) * D_n ** -0.5)
+    w_uv = _bf16_exact(rng.standard_normal((H, D_c, D_v)) * D_c ** -0.5)
+    o_lat = rng.standard_normal((rows, D_c)).astype(np.float32)
+    q_in = torch.zeros(rows, D_n + pad, dtype=torch.bfloat16, device=dev)
+    q_in[:, :D_n] = _t(q_nope, torch.bfloat16)
+    o_in = torch.zeros(rows, D_c + pad, device=dev)
+    o_in[:, :D_c] = _t(o_lat)
+    q_lat = torch.full((rows, D_c), float("nan"), device=dev)
+    kdv.kdv_absorb_q(H, q_in[:, :D_n], _t(w_uk, torch.bfloat16), q_lat)
+    out = torch.full((rows, D_v), float("nan"), device=dev)
+    kdv.kdv_unabsorb_o(H, o_in[:, :D_c], _t(w_uv, torch.bfloat16), out)
+    torch.cuda.synchronize()
+    assert _rel_err(q_lat.cpu().numpy(), oracle.absorb_q(H, q_nope, w_uk)) < 2e-5
+    assert _rel_err(out.cpu().numpy(), oracle.unabsorb_o(H, o_lat, w_uv)) < 2e-5
+
+
 def test_tiny_layer_end_to_end_fp32():
     """The tiny fp32 layer through the GPU: absorb, verify (SIMT), up-project,
     against the oracle's non-absorbed MLA (explicit K = c_kv W_UK, V = c_kv W_UV)."""
