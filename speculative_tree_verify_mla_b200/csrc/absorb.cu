@@ -331,7 +331,7 @@ __device__ __forceinline__ void stage_rows_vec(void* dst, const void* src, int d
 // accumulate in the two halves of a float2 and are added at the end.
 __global__ void __launch_bounds__(P_THREADS)
 absorb_q_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per_head, int32_t H, int32_t D_c,
-                    int32_t D_n, const void* __restrict__ q_nope, int64_t q_stride, int q_dtype, int q_vec,
+                    int32_t D_n, const void* __restrict__ q_nope, int64_t q_stride, int q_dtype,
                     void* __restrict__ q_lat, int64_t o_stride, int o_dtype) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) unsigned long long bar;
@@ -353,8 +353,9 @@ absorb_q_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per
   for (int tb0 = 0; tb0 < rows_per_head; tb0 += PA_TB) {
     const int nr = min(PA_TB, rows_per_head - tb0);
     __syncthreads();                                 // barrier init seen; s_q free
-    if (q_vec) stage_rows_vec<false>(s_q, q_nope, q_dtype, q_stride, tb0, nr, H, h, D_n);
-    else stage_rows(s_q, q_nope, q_dtype, q_stride, tb0, nr, H, h, D_n, P_THREADS);
+    // element-wise: a few loads per thread already fit one round trip, and
+    // the 16-byte form costs registers that this kernel's FMAs need
+    stage_rows(s_q, q_nope, q_dtype, q_stride, tb0, nr, H, h, D_n, P_THREADS);
     __syncthreads();
     if (!landed) {
       ok = wait_landed(b);
@@ -575,8 +576,7 @@ kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32
                  CU_TENSOR_MAP_SWIZZLE_128B)) {
     const dim3 g2((unsigned)((d_latent + PA_ROWS - 1) / PA_ROWS), (unsigned)num_heads);
     absorb_q_tma_kernel<<<g2, P_THREADS, absorb_tma_smem(d_nope), s>>>(
-        tmap, rows / num_heads, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_dtype,
-        (reinterpret_cast<uintptr_t>(q_nope) & 15) == 0 && q_nope_stride % 8 == 0 ? 1 : 0, q_lat, q_lat_stride,
+        tmap, rows / num_heads, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_dtype, q_lat, q_lat_stride,
         out_dtype);
     return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
   }
