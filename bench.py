@@ -45,6 +45,8 @@ KV_ROW_BYTES = 576 * 2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "verify_tc_traffic.json")
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+# NVIDIA's dense (no 2:4 sparsity) B200 figures, reported beside the measured ones
+DATASHEET_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 
 
 def workload_case(layer: int):
@@ -110,6 +112,15 @@ def load_peaks():
                 "hbm_gbs": float(pk["hbm_gbs"]), "source": "measured"}
     except Exception:
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"], source="fallback")
+
+
+def tensor_fracs(tflops: float, peaks) -> dict:
+    """A tensor-bound kernel's rate against the sustained (power-capped)
+    measured bf16 peak and against the datasheet's dense bf16 peak."""
+    return {"frac_of_sustained": tflops / peaks["bf16_tflops_sustained"],
+            "peak_sustained": peaks["bf16_tflops_sustained"],
+            "frac_of_datasheet": tflops / DATASHEET_PEAKS["bf16_tflops"],
+            "peak_datasheet": DATASHEET_PEAKS["bf16_tflops"]}
 
 
 TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 3: ("verify_tc_kernel", "verify_tc.cu"),
@@ -624,7 +635,8 @@ def run_gpu(args):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tc_tflops / peaks["bf16_tflops"], "traffic": traffic,
                      "us_per_launch": tc_us, "flops_per_launch": flops,
-                     "kv_bytes_per_launch": kv_bytes, "peak_source": peaks["source"] + " burst bf16"},
+                     "kv_bytes_per_launch": kv_bytes, "peak_source": peaks["source"] + " burst bf16",
+                     **tensor_fracs(tc_tflops, peaks)},
         "e2e": {"value": e2e_ms * 1e3 / n_calls, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": args.steps * prob.launches_per_step(),

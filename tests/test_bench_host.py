@@ -1,0 +1,31 @@
+"""Host-side pieces of bench.py that need no GPU: the peak table and the
+roofline fractions reported beside the measured one."""
+import json
+
+import pytest
+
+import bench
+
+
+def test_load_peaks_reads_measured_file(tmp_path, monkeypatch):
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"bf16_tflops": 1647.8, "bf16_tflops_sustained": 1344.1, "hbm_gbs": 6543.4}))
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(f))
+    pk = bench.load_peaks()
+    assert pk == {"bf16_tflops": 1647.8, "bf16_tflops_sustained": 1344.1, "hbm_gbs": 6543.4,
+                  "source": "measured"}
+
+
+def test_load_peaks_falls_back_when_missing(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
+    pk = bench.load_peaks()
+    assert pk["source"] == "fallback"
+    assert pk["bf16_tflops"] == pk["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+
+
+def test_tensor_fracs():
+    pk = {"bf16_tflops": 1647.8, "bf16_tflops_sustained": 1344.1, "hbm_gbs": 6543.4}
+    fr = bench.tensor_fracs(672.05, pk)
+    assert fr["frac_of_sustained"] == pytest.approx(0.5)
+    assert fr["frac_of_datasheet"] == pytest.approx(672.05 / 2250.0)
+    assert fr["peak_sustained"] == 1344.1 and fr["peak_datasheet"] == 2250.0
