@@ -256,6 +256,30 @@ def test_absorb_unabsorb_match_einsum():
     np.testing.assert_allclose(out, ref2, rtol=1e-12, atol=1e-12)
 
 
+def test_projections_one_hot_select_weight_columns():
+    """Closed forms of the per-head projections (node-major rows, head =
+    row % H): a one-hot q_nope at k makes q_lat the k-th column of W_UK[h];
+    a one-hot o_lat at d makes the output the d-th row of W_UV[h]. A
+    transposed weight or a node-major/head-major mix-up fails this."""
+    rng = np.random.default_rng(11)
+    H, D_c, D_n, D_v, T = 3, 10, 4, 5, 4
+    rows = T * H
+    w_uk = rng.standard_normal((H, D_c, D_n)).astype(np.float32)
+    w_uv = rng.standard_normal((H, D_c, D_v)).astype(np.float32)
+    ks = rng.integers(0, D_n, rows)
+    ds = rng.integers(0, D_c, rows)
+    q_nope = np.zeros((rows, D_n), np.float32)
+    q_nope[np.arange(rows), ks] = 1.0
+    o_lat = np.zeros((rows, D_c))
+    o_lat[np.arange(rows), ds] = 1.0
+    ql = oracle.absorb_q(H, q_nope, w_uk)
+    out = oracle.unabsorb_o(H, o_lat, w_uv)
+    for row in range(rows):
+        t, h = divmod(row, H)
+        assert np.array_equal(ql[row], w_uk[h][:, ks[row]].astype(np.float64))
+        assert np.array_equal(out[row], w_uv[h][ds[row], :].astype(np.float64))
+
+
 # --------------------------------------------------------------------------
 # closed forms and invariants
 # --------------------------------------------------------------------------
