@@ -186,6 +186,17 @@ def test_library_has_no_oracle_dependency():
                 assert "kdv_oracle" not in txt, fn
 
 
+def test_oracle_has_no_cuda_path_dependency():
+    """The oracle shares no code with the CUDA path: its sources never import
+    the package, load libkdv or include the library's headers."""
+    odir = os.path.join(ROOT, "oracle")
+    for fn in os.listdir(odir):
+        if fn.endswith((".py", ".cpp", ".c", ".h")):
+            txt = open(os.path.join(odir, fn)).read()
+            assert "speculative_tree_verify_mla_b200" not in txt, fn
+            assert "libkdv.so" not in txt and "kdv.h" not in txt and "csrc" not in txt, fn
+
+
 def test_projection_validation(lib):
     fa, fu = lib.kdv_absorb_q, lib.kdv_unabsorb_o
     B, F = kdv.KDV_BF16, kdv.KDV_F32
