@@ -673,7 +673,7 @@ def run_gpu(args):
     return 0
 
 
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -689,9 +689,14 @@ def main():
                          + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
                          + "; paged: " + WORKLOADS["paged"])
     ap.add_argument("--sweep-L", type=int, choices=SWEEP_L, default=5553)
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     args.impl_code = {"tc2": 2, "tc1": 3, "tc2s": 4}[args.kernel]
     args.warmup = max(3, args.warmup)
+    return args
+
+
+def main():
+    args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

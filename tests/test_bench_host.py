@@ -29,3 +29,12 @@ def test_tensor_fracs():
     assert fr["frac_of_sustained"] == pytest.approx(0.5)
     assert fr["frac_of_datasheet"] == pytest.approx(672.05 / 2250.0)
     assert fr["peak_sustained"] == 1344.1 and fr["peak_datasheet"] == 2250.0
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun every rank but 0 leaves the reference arm at once,
+    without work or output (and without touching a process group)."""
+    monkeypatch.setattr(bench, "dist_env", lambda: (2, 1, 1))
+    args = bench.parse_args(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"])
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
