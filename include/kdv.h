@@ -299,6 +299,12 @@ KDV_API kdv_status kdv_tree_accept(const kdv_accept_params* p, void* stream);
  * the first D_c columns of kdv_verify_attn's q rows (q_lat_stride = D_c +
  * D_r). Accumulation is fp32. Limits: D_n <= 512, D_c <= 4096 (absorb);
  * D_c <= 512, D_v <= 4096 (unabsorb); otherwise KDV_ERR_UNSUPPORTED.
+ * bf16 weights with a 16-byte aligned base and rows a multiple of 16 bytes
+ * (D_n resp. D_v a multiple of 8) take the TMA-staged kernels; anything else
+ * takes the general kernels, with the same results up to fp32 summation
+ * order. The TMA-staged kernels wait at most 2 s for their weight tile; if it
+ * never lands they write NaN to their outputs (these entry points take no
+ * device error flag).
  */
 KDV_API kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope,
                                 const void* q_nope, int64_t q_nope_stride, int32_t q_dtype, const void* w_uk,
