@@ -12,7 +12,10 @@ draft tree): kdv_tree_mask_build once, then kdv_verify_attn per layer
 graph of the step; the metric is microseconds per layer.
 
 Also reported: the dominant kernel's roofline (tensor bound), an end-to-end
-number through the C ABI with host buffers, and the CPU oracle as a baseline.
+number through the C ABI with host buffers, the CPU oracle as a baseline, and
+sub-records for the other configurations -- the 200k-key long context and
+the 8-request paged batch, each with its own roofline -- plus greedy
+acceptance, the two projections and the tree builder.
 
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
 torchrun, each rank runs its own layers (weak scaling, no collective on the
@@ -123,8 +126,7 @@ def tensor_fracs(tflops: float, peaks) -> dict:
             "peak_datasheet": DATASHEET_PEAKS["bf16_tflops"]}
 
 
-TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 3: ("verify_tc_kernel", "verify_tc.cu"),
-             4: ("verify_tc2_kernel", "verify_tc2.cu")}
+TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 4: ("verify_tc2_kernel", "verify_tc2.cu")}
 
 
 def kernel_source_hash(src="verify_tc2.cu"):
@@ -483,6 +485,37 @@ def time_tree_build(dev, stream, budget: int = 32, n_calls: int = 64, reps: int 
     return res
 
 
+def time_config(name: str, dev, stream, peaks, impl_code: int = 2, reps: int = 20):
+    """One of the other verify configurations as a sub-record of the headline
+    line: the whole kdv_verify_attn call (kernel + split merge) and the
+    tensor-core kernel alone (the partials-out twin, same grid), each from a
+    CUDA graph replayed `reps` times, against the roofline of that call.
+    Their KV (230 MB for the 200k layer, ~156 MB for the paged batch) exceeds
+    the 126 MB L2, so back-to-back replays read it from HBM."""
+    import torch
+    prob = Problems(workload_cases(name, 1), impl_code, dev)
+    with torch.cuda.stream(stream):
+        prob.step(stream)
+        prob.tc_only(stream)
+    stream.synchronize()
+    g_step, g_tc = graph_of(prob.step, stream), graph_of(prob.tc_only, stream)
+    call_us = replay_us(g_step, stream, reps)
+    tc_us = replay_us(g_tc, stream, reps)
+    del g_step, g_tc
+    err = int(prob.d_err.item())
+    c = prob.cases[0]
+    flops, kv_bytes = case_flops_bytes(c)
+    roof_us = max(flops / (peaks["bf16_tflops"] * 1e12), kv_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+    tc_tflops = flops / (tc_us * 1e-6) / 1e12
+    return {"workload": workload_name(name), "description": WORKLOADS[name],
+            "us_per_call": call_us, "roofline_us": roof_us, "frac_of_roofline": roof_us / call_us,
+            "kernel": {"name": TC_KERNEL[impl_code][0], "us_per_launch": tc_us, "achieved_tflops": tc_tflops,
+                       "peak_tflops": peaks["bf16_tflops"], "frac": tc_tflops / peaks["bf16_tflops"]},
+            "flops_per_call": flops, "kv_bytes_per_call": kv_bytes, "splits": prob.splits[0],
+            "grid_items": prob.items[0], "d_err": err,
+            "timing": f"CUDA graph of one call, {reps} replays, CUDA events on the launch stream"}
+
+
 def run_gpu(args):
     import torch
     from speculative_tree_verify_mla_b200 import kdv
@@ -643,7 +676,9 @@ def run_gpu(args):
         "clocks": clocks,
     }
 
-    if args.workload == "kimi" and rank == 0:
+    if args.workload == "kimi" and rank == 0 and not args.headline_only:
+        result["long_context"] = time_config("long", dev, stream, peaks)
+        result["paged"] = time_config("paged", dev, stream, peaks)
         result["tree_accept"] = time_tree_accept(dev, stream, peaks)
         result["projections"] = time_projections(dev, stream, peaks)
         result["tree_build"] = time_tree_build(dev, stream)
@@ -681,16 +716,18 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT)
     ap.add_argument("--impl", choices=["kdv", "reference"], default="kdv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["tc2", "tc1", "tc2s"], default="tc2",
-                    help="tensor-core kernel: 2-SM MMAs (default), 1-SM MMAs, or 2-SM over a staged "
+    ap.add_argument("--kernel", choices=["tc2", "tc2s"], default="tc2",
+                    help="tensor-core kernel: 2-SM MMAs (default), or the same over a staged "
                          "contiguous copy of a paged pool")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kimi",
                     help="kimi (default, the headline): " + WORKLOADS["kimi"] + "; sweep: "
                          + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
                          + "; paged: " + WORKLOADS["paged"])
     ap.add_argument("--sweep-L", type=int, choices=SWEEP_L, default=5553)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the sub-records (other configurations, acceptance, projections, builder)")
     args = ap.parse_args(argv)
-    args.impl_code = {"tc2": 2, "tc1": 3, "tc2s": 4}[args.kernel]
+    args.impl_code = {"tc2": 2, "tc2s": 4}[args.kernel]
     args.warmup = max(3, args.warmup)
     return args
 

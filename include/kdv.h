@@ -64,10 +64,15 @@ typedef enum {
 #define KDV_DERR_BAD_SLOT 2    /* page_table entry outside [0, num_slots)   */
 #define KDV_DERR_BAD_LENGTH 3  /* device prefix_len differs from host copy  */
 #define KDV_DERR_BAD_TOKEN 4   /* tree-accept: token id out of range        */
-#define KDV_DERR_TIMEOUT 5     /* a bounded in-kernel wait ran out (~1 s);
-                                  the kernel stopped early, output invalid  */
+#define KDV_DERR_TIMEOUT 5     /* a bounded in-kernel wait ran out (1 s or
+                                  wait_limit_ns); the kernel stopped early,
+                                  its outputs are not valid                 */
 #define KDV_DERR_BAD_SCORE 6   /* tree build: a NaN candidate log-probability
                                   (read as -inf)                            */
+#define KDV_DERR_RANGE 7       /* verify (TC kernel): a c_kv value that P.V
+                                  reads has |x| >= 65536, inf or NaN; it is
+                                  outside fp16, the P.V operand type, and
+                                  the affected outputs are not valid        */
 
 /* Element type of q and kv. */
 #define KDV_BF16 0
@@ -75,9 +80,14 @@ typedef enum {
 
 /* Kernel family for kdv_verify_attn. AUTO picks the tensor-core kernel when
  * its shape constraints hold (bf16, d_latent=512, d_rope=64), else SIMT. TC
- * runs 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per work item) and
- * reads a paged pool with TMA four-row gathers; TC_1SM is the 1-SM-MMA
- * variant (2-CTA clusters, 128 rows, contiguous KV only). */
+ * runs 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per work item):
+ * Q.K^T in bf16, P.V with P and V in fp16 (11 significant bits, so the
+ * rounding of the softmax numerators costs ~1.3e-4 of the output's RMS
+ * instead of ~1e-3 in bf16). The c_kv values it reads must therefore lie in
+ * fp16's range, |x| < 65536 (KDV_DERR_RANGE otherwise); rows past a
+ * request's last key are never read. A paged pool is read with TMA four-row
+ * gathers (keys) and per-row loads (values). Value 3 (a 1-SM-MMA variant of
+ * earlier versions) is retired and returns KDV_ERR_UNSUPPORTED. */
 #define KDV_IMPL_AUTO 0
 #define KDV_IMPL_SIMT 1
 #define KDV_IMPL_TC 2
@@ -141,7 +151,7 @@ typedef struct kdv_verify_params {
   int32_t d_rope;        /* D_r: 64 for the TC kernel; 0..64 for SIMT            */
   float scale;           /* softmax scale on q.k (e.g. 1/sqrt(d_nope + d_rope))  */
   int32_t dtype;         /* KDV_BF16 or KDV_F32 (q and kv)                       */
-  int32_t impl;          /* KDV_IMPL_AUTO / _SIMT / _TC                          */
+  int32_t impl;          /* KDV_IMPL_AUTO / _SIMT / _TC / _TC_STAGED             */
   const void* q;         /* [sumT*H][q_row_stride], row = q_lat || q_rope        */
   int64_t q_row_stride;  /* elements between q rows; 0 means D_c + D_r           */
   const void* kv;        /* pool [num_slots][D_c + D_r], row = c_kv || k_rope    */
@@ -162,6 +172,13 @@ typedef struct kdv_verify_params {
   void* workspace;       /* caller-owned scratch, >= kdv_verify_attn_workspace   */
   size_t workspace_bytes;
   int32_t* d_err;        /* nullable device error flag                           */
+  uint64_t wait_limit_ns;  /* TC kernel: how long one pipeline wait inside the
+                              kernel may take before the kernel gives up with
+                              KDV_DERR_TIMEOUT (0 = 1 s). Every wait is
+                              bounded; on giving up, the kernel still retires
+                              its copies and MMAs in flight (waiting up to 1 s
+                              for them) and exits normally, its outputs not
+                              valid. A small value is for testing that path. */
 } kdv_verify_params;
 
 /* Bytes of workspace kdv_verify_attn needs for these parameters (the plan
@@ -181,8 +198,9 @@ KDV_API kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* spl
  * Absorbed Q.K^T over D_c + D_r dims, online softmax, P.V over the D_c latent
  * dims (V is the c_kv part of the same pool row), optional per-split LSE and
  * the split merge. Output o_lat is fp32 [sumT*H][D_c]; lse is the natural-log
- * log-sum-exp of the scaled logits. Requirements: q, kv 16-byte aligned;
- * q_row_stride*elem and (D_c+D_r)*elem multiples of 16 bytes for the TC kernel.
+ * log-sum-exp of the scaled logits. Requirements for the TC kernel: q, kv,
+ * o and o_part 16-byte aligned; q_row_stride*elem and (D_c+D_r)*elem
+ * multiples of 16 bytes (KDV_ERR_INVALID_ARG otherwise).
  */
 KDV_API kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream);
 
@@ -202,6 +220,9 @@ KDV_API kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream);
  *     fewer splits or fewer requests per call fit).
  *   - The first call on a device looks up the array's device address with
  *     the device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a
+ *     cudaDeviceReset of that device it is stale, so do not call this entry
+ *     point on a device that has been reset.
  *   - All calls share the one array and it keeps the previous call's
  *     contents (every byte a call reads, the same call writes first). Calls
  *     whose work overlaps on the GPU race on it: issue them on one stream or

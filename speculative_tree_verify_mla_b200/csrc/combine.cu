@@ -4,8 +4,9 @@
 // reference [1] (one kernel for the long prefix, another for the small tree
 // tail), generalised to any number of key splits: with per-split results
 // (o_k, lse_k), LSE = ln sum_k exp(lse_k) and o = sum_k exp(lse_k - LSE) o_k.
-// HBM-bound: it reads S*(d+1) floats and writes d+1 floats per row. One CTA
-// per row.
+// HBM-bound: it reads S*(d+1) partial values and writes d+1 floats per row.
+#include <cuda_fp16.h>
+
 #include "kdv_internal.cuh"
 
 namespace kdv {
@@ -106,6 +107,107 @@ combine_plan_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws
   }
 }
 
+// The internal merge of the tensor-core kernel's fp16 partials (d = 512):
+// one warp per row, lane l owning columns [16l, 16l+16). The loads of the
+// first eight splits are issued before the split LSEs are reduced, so a
+// row with S <= 8 costs about one memory round trip.
+constexpr int W16_WARPS = 4;
+constexpr int W16_KB = 8;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ void fma_half8(float (&acc)[16], int base, float w, uint4 x) {
+  const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    acc[base + 2 * i] = fmaf(w, f.x, acc[base + 2 * i]);
+    acc[base + 2 * i + 1] = fmaf(w, f.y, acc[base + 2 * i + 1]);
+  }
+}
+
+__global__ void __launch_bounds__(32 * W16_WARPS)
+combine_plan_f16_kernel(const __half* __restrict__ ws_o, const float* __restrict__ ws_lse,
+                        const VerifyPlan p, float* __restrict__ o, float* __restrict__ lse) {
+  constexpr int D = 512;
+  const int lane = threadIdx.x & 31;
+  for (int64_t row = (int64_t)blockIdx.x * W16_WARPS + (threadIdx.x >> 5); row < p.total_rows;
+       row += (int64_t)gridDim.x * W16_WARPS) {
+    int b = 0;
+    while (b + 1 < p.B && (int64_t)p.tree_base[b + 1] * p.H <= row) ++b;
+    const int64_t rows_b = (int64_t)p.T[b] * p.H;
+    const int64_t first = p.part_base[b] + (row - (int64_t)p.tree_base[b] * p.H);
+    const int S = p.S[b];
+    const __half* col0 = ws_o + first * D + lane * 16;
+    uint4 x[W16_KB][2];
+#pragma unroll
+    for (int u = 0; u < W16_KB; ++u)
+      if (u < S) {
+        const uint4* src = reinterpret_cast<const uint4*>(col0 + (int64_t)u * rows_b * D);
+        x[u][0] = __ldg(src);
+        x[u][1] = __ldg(src + 1);
+      }
+    float m = -INFINITY;
+    for (int k = lane; k < S; k += 32) m = fmaxf(m, __ldg(ws_lse + first + (int64_t)k * rows_b));
+    m = warp_max(m);
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    float LSE = -INFINITY;
+    if (m != -INFINITY) {
+      float z = 0.f;
+      for (int k = lane; k < S; k += 32) {
+        const float lk = __ldg(ws_lse + first + (int64_t)k * rows_b);
+        z += lk == -INFINITY ? 0.f : expf(lk - m);
+      }
+      LSE = m + logf(warp_sum(z));
+      for (int k0 = 0; k0 < S; k0 += 32) {
+        const int kk = k0 + lane;
+        const float lk = kk < S ? __ldg(ws_lse + first + (int64_t)kk * rows_b) : -INFINITY;
+        const float wk = lk == -INFINITY ? 0.f : expf(lk - LSE);
+        const int n = min(32, S - k0);
+        for (int j = 0; j < n; j += W16_KB) {
+          if (k0 + j > 0) {      // the first batch was loaded above
+#pragma unroll
+            for (int u = 0; u < W16_KB; ++u)
+              if (j + u < n) {
+                const uint4* src = reinterpret_cast<const uint4*>(col0 + (int64_t)(k0 + j + u) * rows_b * D);
+                x[u][0] = __ldg(src);
+                x[u][1] = __ldg(src + 1);
+              }
+          }
+#pragma unroll
+          for (int u = 0; u < W16_KB; ++u) {
+            const float w = __shfl_sync(0xffffffffu, wk, (j + u) & 31);
+            if (j + u < n) {
+              fma_half8(acc, 0, w, x[u][0]);
+              fma_half8(acc, 8, w, x[u][1]);
+            }
+          }
+        }
+      }
+    }
+    float* orow = o + row * D + lane * 16;
+    if ((reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+      float4* dst = reinterpret_cast<float4*>(orow);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) orow[i] = acc[i];
+    }
+    if (lane == 0 && lse != nullptr) lse[row] = LSE;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, int32_t S,
@@ -117,11 +219,20 @@ cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine_plan(const float* ws_o, const float* ws_lse, const VerifyPlan& p,
+cudaError_t launch_combine_plan(const void* ws_o, const float* ws_lse, const VerifyPlan& p,
                                 int32_t d, float* o, float* lse, cudaStream_t stream) {
   if (p.total_rows == 0) return cudaSuccess;
+  if (p.part_f16) {
+    if (d != 512) return cudaErrorInvalidValue;
+    const int64_t blocks = (p.total_rows + W16_WARPS - 1) / W16_WARPS;
+    const int64_t grid = blocks < (int64_t)1 << 30 ? blocks : (int64_t)1 << 30;
+    combine_plan_f16_kernel<<<(unsigned)grid, 32 * W16_WARPS, 0, stream>>>(static_cast<const __half*>(ws_o), ws_lse,
+                                                                            p, o, lse);
+    return cudaGetLastError();
+  }
   const int64_t grid = p.total_rows < (int64_t)1 << 30 ? p.total_rows : (int64_t)1 << 30;
-  combine_plan_kernel<<<(unsigned)grid, THREADS, 0, stream>>>(ws_o, ws_lse, p, d, o, lse);
+  combine_plan_kernel<<<(unsigned)grid, THREADS, 0, stream>>>(static_cast<const float*>(ws_o), ws_lse, p, d, o,
+                                                              lse);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,7 @@ bool tc_shape_ok(const kdv_verify_params* p) {
   return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64;
 }
 
-bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_1SM || impl == KDV_IMPL_TC_STAGED; }
+bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED; }
 // the 2-SM kernel, reading the pool directly or a staged copy
 bool is_tc2(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED; }
 
@@ -51,6 +51,7 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->num_heads < 1) return KDV_ERR_INVALID_ARG;
   if (p->dtype != KDV_BF16 && p->dtype != KDV_F32) return KDV_ERR_INVALID_ARG;
   if (p->impl < KDV_IMPL_AUTO || p->impl > KDV_IMPL_TC_STAGED) return KDV_ERR_INVALID_ARG;
+  if (p->impl == KDV_IMPL_TC_1SM) return KDV_ERR_UNSUPPORTED;   // retired 1-SM-MMA variant
   if (p->d_latent < 1 || p->d_rope < 0) return KDV_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return KDV_ERR_INVALID_ARG;
   if (p->h_prefix_len == nullptr || p->h_tree_T == nullptr) return KDV_ERR_INVALID_ARG;
@@ -64,7 +65,6 @@ kdv_status check_params(const kdv_verify_params* p, int impl) {
   if (p->return_partials && p->num_splits < 1) return KDV_ERR_INVALID_ARG;
   if (is_tc(impl)) {
     if (!tc_shape_ok(p)) return KDV_ERR_UNSUPPORTED;
-    if (p->page_table != nullptr && impl == KDV_IMPL_TC_1SM) return KDV_ERR_UNSUPPORTED;
   } else {
     if (p->d_latent > 512 || p->d_rope > 64) return KDV_ERR_UNSUPPORTED;
   }
@@ -86,9 +86,11 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
   if ((reinterpret_cast<uintptr_t>(p->q) % esz) || (reinterpret_cast<uintptr_t>(p->kv) % esz))
     return KDV_ERR_INVALID_ARG;
   if (is_tc(impl)) {
-    // TMA needs 16-byte aligned bases and row pitches
+    // TMA needs 16-byte aligned bases and row pitches; the epilogue writes
+    // o / o_part rows in 16-byte vectors
     if (!aligned16(p->q) || !aligned16(p->kv)) return KDV_ERR_INVALID_ARG;
     if ((stride * (int64_t)esz) % 16 != 0) return KDV_ERR_INVALID_ARG;
+    if ((p->o && !aligned16(p->o)) || (p->o_part && !aligned16(p->o_part))) return KDV_ERR_INVALID_ARG;
   }
   float* outs[4] = {p->o, p->lse, p->o_part, p->lse_part};
   for (float* f : outs)
@@ -97,6 +99,18 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
 }
 
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Partial rows of a plan (every request's S_b * T_b * H).
+size_t plan_parts(const VerifyPlan& plan) {
+  return (size_t)plan.part_base[plan.B - 1] + (size_t)plan.S[plan.B - 1] * plan.T[plan.B - 1] * plan.H;
+}
+// Bytes of o_k at the start of the workspace (256-aligned), then lse_k fp32.
+size_t merge_o_bytes(const VerifyPlan& plan, int32_t d) {
+  return align256(plan_parts(plan) * (size_t)d * (plan.part_f16 ? 2 : 4));
+}
+size_t merge_region_bytes(const VerifyPlan& plan, int32_t d) {
+  return merge_o_bytes(plan, d) + plan_parts(plan) * sizeof(float);
+}
 
 // KDV_IMPL_TC_STAGED with a page table: the pool rows are first copied to a
 // contiguous staged region of the workspace.
@@ -108,7 +122,7 @@ bool staged_paged(const kdv_verify_params* p, int impl) {
 kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, size_t* ws_bytes) {
   std::memset(plan, 0, sizeof(*plan));
   const int B = p->batch, H = p->num_heads;
-  const int rows_per_tile = is_tc2(impl) ? TC2_ROWS : impl == KDV_IMPL_TC_1SM ? TC_ROWS : SIMT_ROWS;
+  const int rows_per_tile = is_tc2(impl) ? TC2_ROWS : SIMT_ROWS;
   plan->B = B;
   plan->H = H;
   plan->rows_per_tile = rows_per_tile;
@@ -128,16 +142,13 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
 
   // splits per request
   const int sms = device_sm_count();
-  // TC: one item is a 4-CTA (TC_1SM: 2-CTA) cluster; clusters only fit within
+  // TC: one item is a 4-CTA cluster; clusters only fit within
   // a GPC, so one wave is what the occupancy query reports (fallback: the SM
   // count divided by the cluster size). SIMT: 8-warp CTAs, several per SM.
   double target_items = 4.0 * sms;
   if (is_tc2(impl)) {
     const int n = tc2_max_active_clusters();
     target_items = n > 0 ? n : sms / 4;
-  } else if (impl == KDV_IMPL_TC_1SM) {
-    const int n = tc1_max_active_clusters();
-    target_items = n > 0 ? n : sms / 2;
   }
   const int min_keys = is_tc(impl) ? 2 * TC_KEYS : 128;
   // Automatic splits: choose the chunk X (a multiple of SPLIT_ALIGN keys, at
@@ -213,10 +224,12 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   } else if (all_one) {
     plan->out_mode = OUT_DIRECT;
   } else {
+    // the merge's partials: fp16 o_k from the tensor-core kernel (its outputs
+    // are convex combinations of c_kv values, which that kernel already
+    // requires to lie in fp16's range), fp32 from the SIMT kernel
     plan->out_mode = OUT_WORKSPACE;
-    const size_t o_bytes = (size_t)parts * p->d_latent * sizeof(float);
-    const size_t o_al = (o_bytes + 255) & ~(size_t)255;
-    *ws_bytes = o_al + (size_t)parts * sizeof(float);
+    plan->part_f16 = is_tc2(impl) ? 1 : 0;
+    *ws_bytes = merge_region_bytes(*plan, p->d_latent);
   }
   if (staged_paged(p, impl)) {
     // after the merge region: staged row offsets [B+1], then the staged rows
@@ -313,6 +326,7 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
   a.D_r = p->d_rope;
   a.scale = p->scale;
   a.d_err = p->d_err;
+  a.wait_limit_ns = p->wait_limit_ns;
   float* ws_o = nullptr;
   float* ws_l = nullptr;
   if (plan.out_mode == OUT_DIRECT) {
@@ -322,22 +336,14 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.o = p->o_part;
     a.lse = p->lse_part;
   } else {
-    const size_t parts = (size_t)plan.part_base[plan.B - 1] +
-                         (size_t)plan.S[plan.B - 1] * plan.T[plan.B - 1] * plan.H;
-    const size_t o_bytes = parts * p->d_latent * sizeof(float);
     ws_o = static_cast<float*>(p->workspace);
-    ws_l = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + ((o_bytes + 255) & ~(size_t)255));
+    ws_l = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + merge_o_bytes(plan, p->d_latent));
     a.o = ws_o;
     a.lse = ws_l;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (staged_paged(p, impl)) {
-    size_t merge_bytes = 0;
-    if (plan.out_mode == OUT_WORKSPACE) {
-      const size_t parts = (size_t)plan.part_base[plan.B - 1] +
-                           (size_t)plan.S[plan.B - 1] * plan.T[plan.B - 1] * plan.H;
-      merge_bytes = align256(parts * p->d_latent * sizeof(float)) + parts * sizeof(float);
-    }
+    const size_t merge_bytes = plan.out_mode == OUT_WORKSPACE ? merge_region_bytes(plan, p->d_latent) : 0;
     char* region = static_cast<char*>(p->workspace) + align256(merge_bytes);
     int32_t* staged_off = reinterpret_cast<int32_t*>(region);
     void* staged = region + align256((size_t)(plan.B + 1) * sizeof(int32_t));
@@ -350,9 +356,7 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.page_table = nullptr;
     a.kv_off = staged_off;
   }
-  cudaError_t e = is_tc2(impl)              ? launch_verify_tc2(a, plan, s)
-                  : impl == KDV_IMPL_TC_1SM ? launch_verify_tc(a, plan, s)
-                                            : launch_verify_simt(a, plan, p->dtype, s);
+  cudaError_t e = is_tc2(impl) ? launch_verify_tc2(a, plan, s) : launch_verify_simt(a, plan, p->dtype, s);
   if (e != cudaSuccess) return KDV_ERR_CUDA;
   if (plan.out_mode == OUT_WORKSPACE)
     e = launch_combine_plan(ws_o, ws_l, plan, p->d_latent, p->o, p->lse, s);

@@ -19,6 +19,7 @@ struct VerifyPlan {
   int32_t n_items;
   int32_t rows_per_tile;
   int32_t out_mode;        // OUT_DIRECT / OUT_PARTIALS / OUT_WORKSPACE
+  int32_t part_f16;        // OUT_WORKSPACE partials o_k stored as fp16 (TC kernel)
   int32_t total_rows;      // sumT * H
   int32_t item_base[KDV_MAX_BATCH + 1];
   int32_t L[KDV_MAX_BATCH];
@@ -47,8 +48,10 @@ struct VerifyArgs {
   int32_t D_r;
   float scale;
   float* o;          // OUT_DIRECT: [rows][D_c]; OUT_PARTIALS: [S][rows][D_c]; OUT_WORKSPACE: ws
+                     // (fp16 elements there when the plan's part_f16 is set)
   float* lse;        // matching lse array (may be null in OUT_DIRECT)
   int32_t* d_err;
+  uint64_t wait_limit_ns;   // pipeline-wait bound of the TC kernel (0 = its default, 1 s)
 };
 
 // Where the (request b, split s, local row r) result goes, in rows of D_c.
@@ -76,20 +79,19 @@ cudaError_t launch_mask_build(const int32_t* parent, const int32_t* tree_off, in
                               cudaStream_t stream);
 cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t dtype,
                                cudaStream_t stream);
-cudaError_t launch_verify_tc(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
 cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
-// Work items (clusters) of each TC kernel that fit on the device at once,
-// i.e. one wave; 0 when the query fails (no device).
-int tc1_max_active_clusters();
+// Work items (4-CTA clusters) of the TC kernel that fit on the device at
+// once, i.e. one wave; 0 when the query fails (no device).
 int tc2_max_active_clusters();
 cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, int32_t S,
                                    int64_t rows, int32_t d, float* o, float* lse,
                                    cudaStream_t stream);
-cudaError_t launch_combine_plan(const float* ws_o, const float* ws_lse, const VerifyPlan& p,
+// Merges the workspace partials of a plan: fp32 o_k, or fp16 o_k when
+// p.part_f16 (then d must be 512).
+cudaError_t launch_combine_plan(const void* ws_o, const float* ws_lse, const VerifyPlan& p,
                                 int32_t d, float* o, float* lse, cudaStream_t stream);
 
 // TC kernel tile geometry (shared with the planner).
-constexpr int TC_ROWS = 128;   // query rows per work item of the 1-SM-MMA kernel
 constexpr int TC2_ROWS = 256;  // query rows per work item of the 2-SM-MMA kernel
 constexpr int TC_KEYS = 128;   // keys per S / P tile of the tensor-core kernel
 constexpr int SPLIT_ALIGN = 128;  // split boundaries are multiples of this many keys

@@ -21,7 +21,11 @@ static __device__ __align__(256) unsigned char kdv_noalloc_scratch[KDV_NOALLOC_S
 constexpr int kMaxDevices = 64;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (cached).
+// Device address of the scratch array on the current device, looked up on
+// the first call per device and cached for the life of the process (a
+// cudaDeviceReset of the device would leave the cached address stale; the
+// header says so). Concurrent first calls from several host threads all
+// store the same value.
 kdv_status scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {

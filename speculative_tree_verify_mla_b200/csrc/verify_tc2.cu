@@ -1,7 +1,7 @@
 // verify_tc2.cu -- tensor-core tree-verify MLA attention on 2-SM MMAs
 // (tcgen05.mma cta_group::2, TMEM accumulators, TMA-staged operands).
 //
-// Same operation as verify_tc.cu (page "The Architecture of Diagnosis",
+// The operation (page "The Architecture of Diagnosis",
 // section "Phase 1: Custom CUDA Kernels", item 2; latent dims from page "From
 // Diagnosis to Deployment", section "The Second Thread"): per query row,
 // s_j = scale (q_lat . c_kv[j] + q_rope . k_rope[j]), a softmax over the keys
@@ -16,27 +16,49 @@
 // One work item = 256 query rows of one request and one key split, on a
 // 4-CTA cluster:
 //   CTA 0 + CTA 1 ("S pair"): S = Q K^T with M=256 (rows 0-127 in CTA 0,
-//     128-255 in CTA 1), N=256 keys, K=576. Each CTA holds its rows' q_lat in
-//     TMEM (256 columns), its S tile in the other 256 columns, q_rope in
-//     shared memory, and stages the KV rows of its half of the keys (128 of
-//     every 256) through a 48 KB x 4 ring. CTA 0 issues the MMAs. Two softmax
-//     warpgroups per CTA (one row per thread, keys 0-127 and 128-255 of the
-//     tile) share the row maximum through shared memory, and each pushes its
-//     bf16 P half to the partner CTA on the O side with st.async.
+//     128-255 in CTA 1), N=256 keys, K=576, both operands in shared memory.
+//     Each CTA keeps its rows' q (q_lat || q_rope, 144 KB) in shared memory
+//     for the whole item and stages the KV rows of its half of the keys (128
+//     of every 256) through a 16 KB x 4 ring, one 64-dim K-block per stage;
+//     the next tile's rows are prefetched into L2 meanwhile. TMEM holds two
+//     S buffers of 256 columns, so the MMAs of tile i+1 (issued by CTA 0)
+//     run while the softmax warps drain tile i. Two softmax warpgroups per
+//     CTA (one row per thread, keys 0-127 and 128-255 of the tile) share the
+//     row maximum through shared memory, and each pushes its fp16 P half to
+//     the partner CTA on the O side with st.async.
 //   CTA 2 + CTA 3 ("O pair"): O += P V with M=256, N=256 (two MMAs per 16
 //     keys), K=16, per 128-key P tile. O (128 rows x 512 fp32) fills each
 //     CTA's TMEM; each CTA stages 256 of the 512 V dims (the half of each
-//     N=256 column range the MMA expects from it) through a 16 KB x 8 ring.
-//     CTA 2 issues the MMAs.
+//     N=256 column range the MMA expects from it) through a 16 KB x 6 ring.
+//     Each CTA's producer warp brings its V blocks in with TMA (tiled boxes,
+//     or four-row gathers through a page table), and four converter warps
+//     then re-encode each landed stage in place from bf16 to fp16 (see
+//     below), writing zeros for keys past the split's end so that nothing
+//     of the rows beyond it reaches P.V. CTA 2 issues the MMAs.
+//
+// Precision of P.V. The softmax numerators P are rounded to a 16-bit type
+// before the P.V MMA, and that rounding is the kernel's dominant error. In
+// bf16 (8 significant bits) it leaves a normalised mean error near 1e-3 of
+// the output's RMS; in fp16 (11 bits) about 1.3e-4. A kind::f16 MMA takes A
+// and B of one type, so V is staged as fp16 too: bf16 -> fp16 is exact for
+// every latent value with 2^-14 <= |x| < 65536 (both types keep the 8
+// significant bits), rounds smaller values to fp16 subnormals (an absolute
+// error below 2^-25), and cannot represent |x| >= 65536, which the
+// converters report as KDV_DERR_RANGE. P is at most 2^TAU = 256 by the lazy
+// rescale rule, well inside fp16's range.
 //
 // Every MMA is N=256: with the TMA stream running beside it, N=128 MMAs on
 // this part leave ~35 cycles per instruction unhidden, N=256 ones do not
 // (measured). Cross-CTA arrivals are relaxed (see arrive_on).
 //
-// Softmax, lazy rescale, bounded waits and the split epilogue are as in
-// verify_tc.cu.
+// Softmax: one query row per thread; the running max moves only when a
+// tile's max exceeds it by more than TAU (in log2 units), and then O is
+// rescaled on the O side before the next P tile ("lazy rescale"). Every wait
+// is bounded (TIMEOUT_NS, then KDV_DERR_TIMEOUT and an orderly exit). The
+// split epilogue writes o = O / l and lse = ln 2 * (m + log2 l).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cstring>
@@ -59,13 +81,8 @@ constexpr int KBLOCK_BYTES = HKEYS * 128;           // 128 keys x 64 dims, swizz
 constexpr int VBLOCK_BYTES = VKEYS * 128;           // 32 keys x 64 dims (4 KB)
 constexpr int QBLOCK_BYTES = ROWS * 128;            // 128 rows x 64 dims (16 KB)
 constexpr int QK_BLOCKS = DQ / 64;                  // 9 (8 latent + 1 rope)
-constexpr int QLAT_BLOCKS = 8;
 constexpr int V_LOCAL_BLOCKS = 4;                   // V dim-blocks per O CTA per stage
-constexpr int STAGE_BLOCKS = 3;
-constexpr int KV_STAGES = 4;
-constexpr int KV_STAGE_BYTES = STAGE_BLOCKS * KBLOCK_BYTES;   // 48 KB
-constexpr int Q_STAGES = 3;                         // ring stages covering q_lat staging
-constexpr int STAGES_PER_TILE = QK_BLOCKS / STAGE_BLOCKS;
+constexpr int KV_STAGES = 4;                        // KV ring: one 16 KB K-block per stage
 constexpr int V_STAGES = 6;
 constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
 constexpr int NP = 3;                               // P slots per O CTA
@@ -74,57 +91,61 @@ constexpr int P_KCHUNK_BYTES = ROWS * 16;           // 8 keys of all 128 rows (i
 constexpr int P_MSG_BYTES = P_BYTES + ROWS * 4;
 constexpr int P_SLOT_BYTES = 33792;
 constexpr int STATS_BYTES = 2 * ROWS * 4;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_QLAT_COL = 0;
-constexpr uint32_t TMEM_S_COL = 256;
+constexpr uint32_t TMEM_COLS = 512;               // S side: S buffer b at columns [256 b, 256 b + 256)
 constexpr float TAU = 8.0f;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr uint64_t TIMEOUT_NS = 1000000000ull;
-static_assert(QK_BLOCKS % STAGE_BLOCKS == 0, "stage geometry");
-static_assert(QLAT_BLOCKS * QBLOCK_BYTES <= Q_STAGES * KV_STAGE_BYTES, "q_lat staging");
-static_assert(Q_STAGES < KV_STAGES, "ring too small");
 
 // Shared-memory layout (same offsets in all four CTAs; mapa() relies on it).
-//   S CTAs: [0, 196608) KV ring (4 x 48 KB; q_lat staging in the first 128 KB
-//           at start-up); [196608, 212992) q_rope; row-max / row-sum exchange.
+//   S CTAs: [0, 147456) the CTA's 128 query rows, q_lat || q_rope, as nine
+//           128B-swizzled K-blocks of 64 dims (the A operand of Q.K^T, read
+//           by every tile); [147456, 212992) KV ring (4 x 16 KB, one K-block
+//           of the CTA's 128 keys per stage); row-max / row-sum exchange.
 //   O CTAs: [0, 98304) V ring (6 x 16 KB); 3 P slots; final stats.
-constexpr int OFF_RING = 0;
-constexpr int OFF_QROPE = KV_STAGES * KV_STAGE_BYTES;
-constexpr int OFF_XCHG = OFF_QROPE + QBLOCK_BYTES;           // float [2][2][128] + [128] (S side)
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + QK_BLOCKS * QBLOCK_BYTES;
+constexpr int OFF_XCHG = OFF_KV + KV_STAGES * KBLOCK_BYTES;   // float [2][2][128] + [128] (S side)
 constexpr int XCHG_BYTES = 5 * ROWS * 4;
-constexpr int OFF_P = V_STAGES * V_STAGE_BYTES;
+constexpr int OFF_VRING = 0;
+constexpr int OFF_P = OFF_VRING + V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
 constexpr int OFF_VSLOT = OFF_STATS + STATS_BYTES;            // int32 [256] (O side, paged KV)
 constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
 static_assert(OFF_VSLOT + STILE * 4 <= OFF_MISC, "O-side buffers overlap misc");
 constexpr int OFF_BAR = OFF_MISC;
-constexpr int NUM_BARS = 48;
+constexpr int NUM_BARS = 56;
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
-constexpr int SMEM_USED = OFF_ABORT + 12;
+// teardown records: [0] some CTA of the cluster aborted (written by that CTA
+// into all four); [1..4] per rescale warp, the first P tile it did not see
+// arrive; [5..8] per rescale warp, whether it saw the row statistics arrive
+constexpr int OFF_TEAR = OFF_ABORT + 4;
+constexpr int SMEM_USED = OFF_TEAR + 9 * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of shared memory");
 
 // Barrier slots (each CTA initialises the slots its role uses).
-// S pair. KV_FULL, S_EMPTY, QROPE_FULL and Q_READY are used in CTA 0 only
-// (the MMA issuer's barriers); the others in both S CTAs.
+// S pair. KV_FULL, S_EMPTY and Q_FULL are used in CTA 0 only (the MMA
+// issuer's barriers; both CTAs' bytes count there); the others in both.
 constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + KV_STAGES, B_S_FULL = B_KV_EMPTY + KV_STAGES,
-              B_S_EMPTY = B_S_FULL + 1, B_P_EMPTY = B_S_EMPTY + 1, B_QLAT_FULL = B_P_EMPTY + NP,
-              B_QROPE_FULL = B_QLAT_FULL + 1, B_Q_READY = B_QROPE_FULL + 1, B_S_DRAIN = B_Q_READY + 1;
-// O pair. V_FULL, READY and O_DRAIN in CTA 2 only.
+              B_S_EMPTY = B_S_FULL + 2, B_P_EMPTY = B_S_EMPTY + 2, B_Q_FULL = B_P_EMPTY + NP,
+              B_S_DRAIN = B_Q_FULL + QK_BLOCKS;
+// O pair. V_FULL, READY and O_DRAIN in CTA 2 only; V_LANDED (a stage's TMA
+// bytes are in this CTA) and V_EMPTY in both.
 constexpr int B_V_FULL = B_S_DRAIN + 1, B_V_EMPTY = B_V_FULL + V_STAGES, B_P_FULL = B_V_EMPTY + V_STAGES,
               B_READY = B_P_FULL + NP, B_PV_DONE = B_READY + NP, B_STATS = B_PV_DONE + NP,
-              B_O_DRAIN = B_STATS + 1;
-static_assert(B_O_DRAIN < NUM_BARS, "barrier slots");
+              B_O_DRAIN = B_STATS + 1, B_V_LANDED = B_O_DRAIN + 1;
+static_assert(B_V_LANDED + V_STAGES <= NUM_BARS, "barrier slots");
 
 constexpr uint16_t S_PAIR = 0x3, O_PAIR = 0xC;     // cluster CTA masks
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(256, 256, false, false);
-constexpr uint32_t IDESC_PV = idesc_bf16_f32(256, 256, false, true);
+constexpr uint32_t IDESC_PV = idesc_f16_f32(256, 256, false, true);   // fp16 P and V
 
 constexpr int THREADS = 384;
 constexpr int WG_FIRST_WARP = 4;      // warps 4-7: softmax keys 0-127 / O-side rescale + epilogue
-constexpr int WG2_FIRST_WARP = 8;     // warps 8-11: softmax keys 128-255 (S side)
+constexpr int WG2_FIRST_WARP = 8;     // warps 8-11: softmax keys 128-255 (S side) / V converters (O side)
+constexpr int CONVERTERS = 4;         // O-side converter warps per CTA
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -136,23 +157,37 @@ struct Ctx {
   uint32_t base;
   volatile uint32_t* abort_flag;
   int32_t* d_err;
+  uint64_t limit;        // ns a pipeline wait may take (drain waits always get TIMEOUT_NS)
   __device__ uint32_t bar(int i) const { return base + OFF_BAR + 8 * i; }
 };
 
+// Bounded wait for phase `parity` of `bar`. A pipeline wait gives up after
+// c.limit ns (recording KDV_DERR_TIMEOUT and raising this CTA's abort flag)
+// or as soon as the flag is up; a drain wait -- one that retires this CTA's
+// own copies and MMAs before it exits -- ignores the flag and waits up to
+// TIMEOUT_NS.
 __device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t lim = drain ? TIMEOUT_NS : c.limit;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (!drain && *c.abort_flag) return false;
-      if (globaltimer() - t0 > TIMEOUT_NS) {
+      if (globaltimer() - t0 > lim) {
         *c.abort_flag = 1;
         record_error(c.d_err, KDV_DERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// Wait for phase `parity` of `bar` until the globaltimer reaches `deadline`.
+__device__ __noinline__ bool wait_until(uint32_t bar, uint32_t parity, uint64_t deadline) {
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer() > deadline) return false;
+  return true;
 }
 
 // Warp-wide bounded wait: lane 0 polls the barrier and the warp then syncs,
@@ -213,6 +248,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   c.base = base;
   c.abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_ABORT);
   c.d_err = a.d_err;
+  c.limit = a.wait_limit_ns > 0 ? a.wait_limit_ns : TIMEOUT_NS;
 
   // ---- work item ---------------------------------------------------------
   const int item = blockIdx.x >> 2;
@@ -234,33 +270,26 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   // ---- setup -------------------------------------------------------------
   if (threadIdx.x == 0) {
     *c.abort_flag = 0;
+    reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR)[0] = 0;
     if (s_side) {
       for (int i = 0; i < KV_STAGES; ++i) {
         mbar_init(c.bar(B_KV_FULL + i), 1);
         mbar_init(c.bar(B_KV_EMPTY + i), 1);
       }
-      mbar_init(c.bar(B_S_FULL), 1);
-      mbar_init(c.bar(B_S_EMPTY), 16);                   // every softmax warp of both S CTAs
-      for (int i = 0; i < NP; ++i) mbar_init(c.bar(B_P_EMPTY + i), 1);
-      mbar_init(c.bar(B_QLAT_FULL), 1);
-      mbar_init(c.bar(B_QROPE_FULL), 1);
-      mbar_init(c.bar(B_Q_READY), 8);                    // the q_lat-copying warps of both S CTAs
-      mbar_init(c.bar(B_S_DRAIN), 1);
-      // KV_FULL phase k of ring stage st belongs to ring use st + 4k; the
-      // stages that hold q_lat at start-up (uses 0-2) carry no KV, so their
-      // first phase is completed here
-      for (int st = 0; st < Q_STAGES; ++st) mbar_arrive(c.bar(B_KV_FULL + st));
-      if (leader) {
-        if (a.prefix_len != nullptr && a.prefix_len[b] != L) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
-        if (a.tree_off != nullptr && a.tree_off[b] != p.tree_base[b]) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
-        if ((int64_t)a.kv_off[b + 1] - kv_base < (int64_t)n_keys) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(c.bar(B_S_FULL + i), 1);
+        mbar_init(c.bar(B_S_EMPTY + i), 16);             // every softmax warp of both S CTAs
       }
+      for (int i = 0; i < NP; ++i) mbar_init(c.bar(B_P_EMPTY + i), 1);
+      for (int i = 0; i < QK_BLOCKS; ++i) mbar_init(c.bar(B_Q_FULL + i), 1);
+      mbar_init(c.bar(B_S_DRAIN), 1);
       tma_prefetch_desc(&tmap_kv);
       tma_prefetch_desc(&tmap_q);
     } else {
       for (int i = 0; i < V_STAGES; ++i) {
-        mbar_init(c.bar(B_V_FULL + i), 1);
+        mbar_init(c.bar(B_V_FULL + i), 2 * CONVERTERS);   // the converter warps of both O CTAs
         mbar_init(c.bar(B_V_EMPTY + i), 1);
+        mbar_init(c.bar(B_V_LANDED + i), 1);
       }
       for (int i = 0; i < NP; ++i) {
         mbar_init(c.bar(B_P_FULL + i), 1);
@@ -285,13 +314,22 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
 
+  if (s_side && leader && warp == 2 && lane == 0) {
+    // device copies of the lengths against the host copies the plan used
+    if (a.prefix_len != nullptr && a.prefix_len[b] != L) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+    if (a.tree_off != nullptr && a.tree_off[b] != p.tree_base[b]) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+    if ((int64_t)a.kv_off[b + 1] - kv_base < (int64_t)n_keys) record_error(a.d_err, KDV_DERR_BAD_LENGTH);
+  }
   if (s_side) {
     // ======================================================= S pair
     if (warp == 0 && (PAGED || lane == 0)) {
-      // ---------------- producer (both S CTAs): q_lat staging (local), q_rope
-      // and this CTA's 128 of every 256 KV rows (counted on the leader's
-      // barriers). Paged KV: the whole warp gathers, 4 rows per lane.
-      const int n_stg = n_stiles * STAGES_PER_TILE;
+      // ---------------- producer (both S CTAs): this CTA's 128 query rows
+      // (nine K-blocks, kept for the whole item) and its 128 of every 256 KV
+      // rows, one K-block per ring stage; everything counts on the leader's
+      // barriers. Contiguous KV: the next tile's rows are prefetched into L2
+      // while this tile streams. Paged KV: the whole warp gathers, 4 rows per
+      // lane.
+      const int n_stg = n_stiles * QK_BLOCKS;
       int issued = 0;
       // paged KV: lane l gathers keys 4l..4l+3 of this CTA's 128; their slots
       // are read one tile ahead so the page-table latency stays off the path
@@ -303,23 +341,23 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       }
       if (n_stiles > 0 && lane == 0) {
         const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
-        mbar_arrive_expect_tx(c.bar(B_QLAT_FULL), QLAT_BLOCKS * QBLOCK_BYTES);
-        for (int blk = 0; blk < QLAT_BLOCKS; ++blk)
-          tma_load_2d(base + OFF_RING + blk * QBLOCK_BYTES, &tmap_q, c.bar(B_QLAT_FULL), blk * 64, qy);
-        if (leader) mbar_arrive_expect_tx(c.bar(B_QROPE_FULL), 2 * QBLOCK_BYTES);
-        tma_load_2d_pair(base + OFF_QROPE, &tmap_q, mapa(c.bar(B_QROPE_FULL), lead_rank), QLAT_BLOCKS * 64, qy);
+        for (int blk = 0; blk < QK_BLOCKS; ++blk) {
+          if (leader) mbar_arrive_expect_tx(c.bar(B_Q_FULL + blk), 2 * QBLOCK_BYTES);
+          tma_load_2d_pair(base + OFF_Q + blk * QBLOCK_BYTES, &tmap_q, mapa(c.bar(B_Q_FULL + blk), lead_rank),
+                           blk * 64, qy);
+        }
       }
       for (int g = 0; g < n_stg; ++g) {
-        const int pos = g + Q_STAGES, st = pos % KV_STAGES;
-        const uint32_t eparity = ((pos / KV_STAGES) & 1) ^ 1;
+        const int st = g % KV_STAGES;
+        const uint32_t eparity = ((g / KV_STAGES) & 1) ^ 1;
         if (!(PAGED ? wait_warp(c, c.bar(B_KV_EMPTY + st), eparity) : wait_bar(c, c.bar(B_KV_EMPTY + st), eparity)))
           break;
-        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KV_STAGE_BYTES);
-        const int tile = g / STAGES_PER_TILE, blk0 = (g % STAGES_PER_TILE) * STAGE_BLOCKS;
+        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
+        const int tile = g / QK_BLOCKS, blk = g % QK_BLOCKS;
         const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
-        const uint32_t dst = base + OFF_RING + st * KV_STAGE_BYTES;
+        const uint32_t dst = base + OFF_KV + st * KBLOCK_BYTES;
         if (PAGED) {
-          if (g % STAGES_PER_TILE == 0) {
+          if (blk == 0) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) slot[q] = nslot[q];
             if (tile + 1 < n_stiles) {
@@ -328,62 +366,51 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
               for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
             }
           }
-          for (int e = 0; e < STAGE_BLOCKS; ++e)
-            tma_gather4_pair(dst + e * KBLOCK_BYTES + lane * 512, &tmap_kv, fb, (blk0 + e) * 64, slot[0], slot[1],
-                             slot[2], slot[3]);
+          tma_gather4_pair(dst + lane * 512, &tmap_kv, fb, blk * 64, slot[0], slot[1], slot[2], slot[3]);
         } else {
           const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
-          for (int e = 0; e < STAGE_BLOCKS; ++e)
-            tma_load_2d_pair(dst + e * KBLOCK_BYTES, &tmap_kv, fb, (blk0 + e) * 64, y);
+          if (blk == 0 && tile + 1 < n_stiles)
+            for (int e = 0; e < QK_BLOCKS; ++e) tma_prefetch_l2(&tmap_kv, e * 64, y + STILE);
+          tma_load_2d_pair(dst, &tmap_kv, fb, blk * 64, y);
         }
         issued = g + 1;
       }
-      if (n_stiles > 0 && lane == 0) wait_bar(c, c.bar(B_QLAT_FULL), 0, true);
       if (leader && lane == 0) {
         // retire copies in flight (both halves count on the leader's barriers)
-        if (n_stiles > 0) wait_bar(c, c.bar(B_QROPE_FULL), 0, true);
-        for (int g = max(0, issued - KV_STAGES); g < issued; ++g) {
-          const int pos = g + Q_STAGES;
-          wait_bar(c, c.bar(B_KV_FULL + pos % KV_STAGES), (pos / KV_STAGES) & 1, true);
-        }
+        if (n_stiles > 0)
+          for (int blk = 0; blk < QK_BLOCKS; ++blk) wait_bar(c, c.bar(B_Q_FULL + blk), 0, true);
+        for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
+          wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
       }
     } else if (warp == 1 && lane == 0 && leader) {
-      // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T
-      bool ok = n_stiles == 0 || (wait_bar(c, c.bar(B_Q_READY), 0) && wait_bar(c, c.bar(B_QROPE_FULL), 0));
-      tc_fence_after();
-      if (ok && n_stiles > 0) {
-        // the q_lat staging stages are free in both S CTAs once Q is in TMEM
-        for (int st = 0; st < Q_STAGES; ++st) {
-          mbar_arrive(c.bar(B_KV_EMPTY + st));
-          mbar_arrive_remote_relaxed(mapa(c.bar(B_KV_EMPTY + st), lead_rank + 1));
-        }
-      }
-      const uint32_t d = tmem + TMEM_S_COL;
+      // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T,
+      // both operands in shared memory, into the two TMEM S buffers in turn:
+      // the MMAs of tile i+1 run while the softmax warps drain tile i. The
+      // first tile waits for each query K-block as it lands.
+      bool ok = true;
       for (int i = 0; ok && i < n_stiles; ++i) {
-        if (!wait_bar(c, c.bar(B_S_EMPTY), (i & 1) ^ 1)) break;
+        const int sb = i & 1;
+        if (!wait_bar(c, c.bar(B_S_EMPTY + sb), ((i >> 1) & 1) ^ 1)) break;
         tc_fence_after();
-        for (int gs = 0; ok && gs < STAGES_PER_TILE; ++gs) {
-          const int pos = i * STAGES_PER_TILE + gs + Q_STAGES, st = pos % KV_STAGES;
-          if (!wait_bar(c, c.bar(B_KV_FULL + st), (pos / KV_STAGES) & 1)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int e = 0; e < STAGE_BLOCKS; ++e) {
-            const int blk = gs * STAGE_BLOCKS + e;
-            const uint32_t kb = base + OFF_RING + st * KV_STAGE_BYTES + e * KBLOCK_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bdesc = sw128_desc(kb + kk * 32, 16, 1024);
-              const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
-              if (blk < QLAT_BLOCKS)
-                mma2_ts(d, tmem + TMEM_QLAT_COL + (blk * 4 + kk) * 8, bdesc, IDESC_QK, acc);
-              else
-                mma2_ss(d, sw128_desc(base + OFF_QROPE + kk * 32, 16, 1024), bdesc, IDESC_QK, acc);
-            }
+        const uint32_t d = tmem + (uint32_t)(sb * 256);
+        for (int blk = 0; blk < QK_BLOCKS; ++blk) {
+          const int g = i * QK_BLOCKS + blk, st = g % KV_STAGES;
+          if ((i == 0 && !wait_bar(c, c.bar(B_Q_FULL + blk), 0)) ||
+              !wait_bar(c, c.bar(B_KV_FULL + st), (g / KV_STAGES) & 1)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t qb = base + OFF_Q + blk * QBLOCK_BYTES;
+          const uint32_t kb = base + OFF_KV + st * KBLOCK_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma2_ss(d, sw128_desc(qb + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), IDESC_QK,
+                    (blk > 0 || kk > 0) ? 1u : 0u);
           tc_commit2_mc(c.bar(B_KV_EMPTY + st), S_PAIR);
         }
         if (!ok) break;
-        tc_commit2_mc(c.bar(B_S_FULL), S_PAIR);
+        tc_commit2_mc(c.bar(B_S_FULL + sb), S_PAIR);
       }
       tc_commit2_mc(c.bar(B_S_DRAIN), (uint16_t)(1u << rank));
       wait_bar(c, c.bar(B_S_DRAIN), 0, true);
@@ -398,31 +425,6 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
       float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);   // [2 parity][2 hw][128] (+ final sums)
       bool ok = true;
-      if (n_stiles > 0 && hw == 0) {
-        // q_lat row (TMA-staged, 128B-swizzled) -> TMEM columns [0, 256)
-        ok = wait_warp(c, c.bar(B_QLAT_FULL), 0);
-        if (__all_sync(0xffffffffu, ok)) {
-#pragma unroll 1
-          for (int blk = 0; blk < QLAT_BLOCKS; ++blk) {
-            uint32_t v[32];
-            const uint8_t* rowp = smem + OFF_RING + blk * QBLOCK_BYTES + r * 128;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 u4 = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (r & 7)) << 4));
-              v[4 * ch + 0] = u4.x;
-              v[4 * ch + 1] = u4.y;
-              v[4 * ch + 2] = u4.z;
-              v[4 * ch + 3] = u4.w;
-            }
-            __syncwarp();
-            tmem_st32(tmem + lane_base + TMEM_QLAT_COL + blk * 32, v);
-          }
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_on(c.bar(B_Q_READY), lead_rank, rank);
-      }
       const uint64_t mask_t = valid ? a.mask[p.tree_base[b] + row / H] : 0ull;
       // a warp whose 32 rows all lie past the request's last row (the tail
       // of its last row tile) sends zeros and does no softmax work
@@ -433,18 +435,18 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const uint32_t pslot0 = mapa(base + OFF_P, o_rank);
       const uint32_t pbar0 = mapa(c.bar(B_P_FULL), o_rank);
       for (int i = 0; i < n_stiles; ++i) {
-        ok = wait_warp(c, c.bar(B_S_FULL), i & 1) && ok;
+        ok = wait_warp(c, c.bar(B_S_FULL + (i & 1)), (i >> 1) & 1) && ok;
         const bool wok = __all_sync(0xffffffffu, ok);
         uint32_t sv[KEYS];
         if (wok) {
           __syncwarp();
           tc_fence_after();
           // one 128-column load: the S half arrives in a single TMEM round trip
-          tmem_ld128(tmem + lane_base + TMEM_S_COL + hw * KEYS, sv);
+          tmem_ld128(tmem + lane_base + (uint32_t)((i & 1) * 256 + hw * KEYS), sv);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) arrive_on(c.bar(B_S_EMPTY), lead_rank, rank);
+          if (lane == 0) arrive_on(c.bar(B_S_EMPTY + (i & 1)), lead_rank, rank);
         } else {
 #pragma unroll
           for (int k = 0; k < KEYS; ++k) sv[k] = 0u;
@@ -515,7 +517,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
               const float p0 = ex2(__uint_as_float(sv[8 * ch + 2 * q]) - m_use);
               const float p1 = ex2(__uint_as_float(sv[8 * ch + 2 * q + 1]) - m_use);
               lsum += p0 + p1;
-              w[q] = pack_bf16x2(p0, p1);
+              w[q] = pack_f16x2(p0, p1);
             }
             // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
             // so a warp's 32 rows fill 512 contiguous bytes per store
@@ -546,10 +548,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
     // ======================================================= O pair
     if (warp == 0 && (PAGED || lane == 0)) {
       // ---------------- V producer (both O CTAs): this CTA's 256 dims of
-      // every 32 keys; local block lb holds dims 64*((lb/2)*4 + half*2 + lb%2).
+      // every 32 keys, landing on this CTA's own V_LANDED barrier; local
+      // block lb holds dims 64*((lb/2)*4 + half*2 + lb%2), bf16, 128B-swizzled.
       // Paged KV: lanes 0-7 gather 4 rows each.
       int issued = 0;
-      const int n_sub = (KEYS / VKEYS) * n_ptiles;
+      const int n_sub = (STILE / VKEYS) * n_stiles;
       // paged KV: the 256 slots of an S tile sit in a shared table (lane l
       // reads keys 8l..8l+7 of the next tile one tile ahead, in registers)
       int32_t* vslot = reinterpret_cast<int32_t*>(smem + OFF_VSLOT);
@@ -563,10 +566,10 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const uint32_t eparity = ((u / V_STAGES) & 1) ^ 1;
         if (!(PAGED ? wait_warp(c, c.bar(B_V_EMPTY + st), eparity) : wait_bar(c, c.bar(B_V_EMPTY + st), eparity)))
           break;
-        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
+        const uint32_t lb_bar = c.bar(B_V_LANDED + st);
+        if (lane == 0) mbar_arrive_expect_tx(lb_bar, V_STAGE_BYTES);
         const int key0 = stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS;
-        const uint32_t dst = base + OFF_RING + st * V_STAGE_BYTES;
-        const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
+        const uint32_t dst = base + OFF_VRING + st * V_STAGE_BYTES;
         if (PAGED) {
           const int vt = u / (STILE / VKEYS);
           if (u % (STILE / VKEYS) == 0) {          // entering S tile vt: publish its slots
@@ -585,8 +588,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             for (int q = 0; q < 4; ++q) slot[q] = vslot[k + q];
             for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
               const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-              tma_gather4_pair(dst + lb * VBLOCK_BYTES + lane * 512, &tmap_v, fb, gb * 64, slot[0], slot[1], slot[2],
-                               slot[3]);
+              tma_gather4(dst + lb * VBLOCK_BYTES + lane * 512, &tmap_v, lb_bar, gb * 64, slot[0], slot[1], slot[2],
+                          slot[3]);
             }
           }
           __syncwarp();
@@ -594,14 +597,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           const int32_t y = (int32_t)(kv_base + key0);
           for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
             const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-            tma_load_2d_pair(dst + lb * VBLOCK_BYTES, &tmap_v, fb, gb * 64, y);
+            tma_load_2d(dst + lb * VBLOCK_BYTES, &tmap_v, lb_bar, gb * 64, y);
           }
         }
         issued = u + 1;
       }
-      if (leader && lane == 0)
+      if (lane == 0)
         for (int u = max(0, issued - V_STAGES); u < issued; ++u)
-          wait_bar(c, c.bar(B_V_FULL + u % V_STAGES), (u / V_STAGES) & 1, true);
+          wait_bar(c, c.bar(B_V_LANDED + u % V_STAGES), (u / V_STAGES) & 1, true);
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------- pair MMA issuer: O[256 x 512] += P[256 x 128] . V[128 x 512]
       for (int i = 0; i < n_ptiles; ++i) {
@@ -613,7 +616,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           const int u = (KEYS / VKEYS) * i + h, st = u % V_STAGES;
           if (!wait_bar(c, c.bar(B_V_FULL + st), (u / V_STAGES) & 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t vst = base + OFF_RING + st * V_STAGE_BYTES;
+          const uint32_t vst = base + OFF_VRING + st * V_STAGE_BYTES;
 #pragma unroll
           for (int kk = 0; kk < VKEYS / 16; ++kk) {
             const int k = (VKEYS / 16) * h + kk;
@@ -656,9 +659,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       bool bad = false;
       if (eh == 0) {
         bool ok = true;
+        int first_miss = n_ptiles;          // first P tile this warp did not see arrive
         for (int i = 0; i < n_ptiles; ++i) {
           const int slot = i % NP;
-          ok = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1) && ok;
+          const bool got = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1);
+          if (!got && first_miss == n_ptiles) first_miss = i;
+          ok = got && ok;
           fence_proxy_async_smem();      // P arrived by st.async; the pair's MMA reads it
           const float al = *reinterpret_cast<volatile float*>(smem + OFF_P + slot * P_SLOT_BYTES + P_BYTES + r * 4);
           const bool need = ok && i > 0 && al != 1.f;
@@ -693,8 +699,57 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           have_o = wait_warp(c, c.bar(B_PV_DONE + i % NP), (i / NP) & 1, !ok);
         }
         have_o = __all_sync(0xffffffffu, have_o);
-        ok = wait_warp(c, c.bar(B_STATS), 0) && ok && have_o == (n_ptiles > 0);
+        const bool got_stats = wait_warp(c, c.bar(B_STATS), 0);
+        ok = got_stats && ok && have_o == (n_ptiles > 0);
         bad = !ok;
+        if (lane == 0) {
+          volatile uint32_t* tear = reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR);
+          tear[1 + sp] = (uint32_t)first_miss;
+          tear[5 + sp] = got_stats ? 1u : 0u;
+        }
+      } else {
+        // ---------------- V converters (warps 8-11, both O CTAs): once stage
+        // u's TMA bytes have landed in this CTA, re-encode its 16 KB in place
+        // from bf16 to fp16 (every 16-byte chunk keeps its place; the chunk at
+        // byte b holds 8 dims of key b % 4096 / 128 of the stage), write
+        // zeros for keys at or past the split's end, and tell the MMA issuer.
+        // Thread t takes chunks t, t + 128, ...: a warp covers 512 contiguous
+        // bytes per access.
+        const int tid = (warp - WG2_FIRST_WARP) * 32 + lane;
+        const int n_sub = (STILE / VKEYS) * n_stiles;
+        const uint32_t vfull_lead = mapa(c.bar(B_V_FULL), lead_rank);
+        uint32_t range = 0;
+        bool ok = true;
+        for (int u = 0; ok && u < n_sub; ++u) {
+          const int st = u % V_STAGES;
+          ok = wait_warp(c, c.bar(B_V_LANDED + st), (u / V_STAGES) & 1);
+          if (!ok) break;
+          const int live = k_hi - (stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS);
+          const uint32_t sb = base + OFF_VRING + st * V_STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < V_STAGE_BYTES / 16 / (32 * CONVERTERS); ++i) {
+            const uint32_t off = (uint32_t)(tid + 32 * CONVERTERS * i) * 16u;
+            const uint32_t addr = sb + off;
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+            if ((int)((off & (VBLOCK_BYTES - 1)) >> 7) < live) {
+              range |= bf16x2_beyond_f16(v.x) | bf16x2_beyond_f16(v.y) | bf16x2_beyond_f16(v.z) |
+                       bf16x2_beyond_f16(v.w);
+              v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+            } else {
+              v = make_uint4(0u, 0u, 0u, 0u);
+            }
+            st_shared_v4(addr, v.x, v.y, v.z, v.w);
+          }
+          // the pair's MMA reads these bytes through the async proxy
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive(c.bar(B_V_FULL + st));
+            else mbar_arrive_remote(vfull_lead + st * 8);
+          }
+        }
+        if (__any_sync(0xffffffffu, range != 0) && lane == 0) record_error(a.d_err, KDV_DERR_RANGE);
       }
       // warps 8-11 learn of the final MMA and the statistics through this barrier
       bad = named_bar_or(1, 2 * 128, bad);
@@ -706,27 +761,47 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const float inv = (l > 0.f && !bad) ? 1.f / l : 0.f;
       const float lse = (l > 0.f && !bad) ? (m + __log2f(l)) * LN2 : -INFINITY;
       const int64_t orow = out_row_index(p, b, split, row);
-      // whole-warp rows go out as 32x32 fp32 boxes through the TMA store
-      // (staged 128B-swizzled in the V ring, free once the last PV is done);
-      // a warp straddling the end of the request stores row by row
+      // Whole-warp rows go out through TMA stores of 4 KB boxes staged
+      // 128B-swizzled in the V ring (free once the last PV is done): 32 rows
+      // x 32 fp32 columns, or, for the internal merge's fp16 partials, 32
+      // rows x 64 fp16 columns. A warp straddling the end of the request
+      // stores row by row.
       const int wrow0 = row0 + sp * 32;
       const bool warp_full = o_tma != 0 && !bad && wrow0 + 32 <= rows_b;
       const int64_t wy = out_row_index(p, b, split, wrow0);
-      const uint32_t stage = base + OFF_RING + ew * 8192;
-      float* orow_ptr = a.o + orow * DC;
+      const uint32_t stage = base + OFF_VRING + ew * 8192;
+      const int cols_per_box = p.part_f16 ? 64 : 32;
 #pragma unroll 1
-      for (int cb = 0; cb < 256 / 32; ++cb) {
-        const int col = eh * 256 + cb * 32;
+      for (int cb = 0; cb < 256 / cols_per_box; ++cb) {
+        const int col = eh * 256 + cb * cols_per_box;
         uint32_t v[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_base + col, v);
-          tmem_wait_ld();
+        if (p.part_f16) {
+          // two 32-column TMEM loads packed into 32 words of fp16 pairs
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t t[32];
+            if (have_o) {
+              tmem_ld32(tmem + lane_base + col + 32 * hf, t);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) t[k] = 0u;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              v[16 * hf + k] = pack_f16x2(__uint_as_float(t[2 * k]) * inv, __uint_as_float(t[2 * k + 1]) * inv);
+          }
         } else {
+          if (have_o) {
+            tmem_ld32(tmem + lane_base + col, v);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = 0u;
+            for (int k = 0; k < 32; ++k) v[k] = 0u;
+          }
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * inv);
         }
-#pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * inv);
         if (warp_full) {
           const uint32_t buf = stage + (cb & 1) * 4096;
           if (cb >= 2) {
@@ -735,9 +810,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         :: "r"(buf + lane * 128 + ((q ^ (lane & 7)) << 4)), "r"(v[4 * q]), "r"(v[4 * q + 1]),
-                            "r"(v[4 * q + 2]), "r"(v[4 * q + 3]) : "memory");
+            st_shared_v4(buf + lane * 128 + ((q ^ (lane & 7)) << 4), v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                         v[4 * q + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -745,11 +819,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             bulk_commit_group();
           }
         } else if (valid) {
+          // 128 bytes of this row: 32 fp32 or 64 fp16 columns
+          uint4* dst = p.part_f16 ? reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.o) + orow * DC + col)
+                                  : reinterpret_cast<uint4*>(a.o + orow * DC + col);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(orow_ptr + col + 4 * q) =
-                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
       }
       if (warp_full && lane == 0) bulk_wait_group_read<0>();
@@ -759,9 +833,36 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   }
 
   // ---- teardown ----------------------------------------------------------
+  // After an abort (a wait that ran out) the O side stops waiting for P
+  // tiles, so st.async bytes from the S pair could still be in flight toward
+  // an O CTA when it reaches this point. So: a CTA whose abort flag is up
+  // tells all four CTAs; after the cluster barrier, if any CTA aborted, each
+  // O CTA waits -- in order, against one deadline -- for every P-tile phase
+  // and the statistics that none of its rescale warps saw arrive, and a
+  // second barrier keeps every CTA resident until then. (Every phase the
+  // drain waits for is at most the barrier's current one: a later phase of
+  // a slot needs the MMAs of this one, which need all rescale warps to have
+  // seen it.) The normal path costs one CTA barrier.
+  volatile uint32_t* tear = reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR);
   __syncwarp();
+  __syncthreads();
+  if (threadIdx.x < 4 && *c.abort_flag != 0) st_cluster_u32(mapa(base + OFF_TEAR, threadIdx.x), 1u);
   tc_fence_before();
   cluster_sync();
+  if (tear[0] != 0) {
+    if (!s_side && threadIdx.x == 0 && n_ptiles > 0) {
+      int from = 0;
+      bool stats = false;
+      for (int w = 0; w < 4; ++w) {
+        from = max(from, (int)tear[1 + w]);
+        stats = stats || tear[5 + w] != 0;
+      }
+      const uint64_t deadline = globaltimer() + TIMEOUT_NS;
+      for (int i = from; i < n_ptiles; ++i) wait_until(c.bar(B_P_FULL + i % NP), (i / NP) & 1, deadline);
+      if (!stats) wait_until(c.bar(B_STATS), 0, deadline);
+    }
+    cluster_sync();
+  }
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc2(tmem, TMEM_COLS);
@@ -803,23 +904,25 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
   };
   CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o;
   const bool paged = a.page_table != nullptr;
-  // paged KV: one map with one-row boxes serves the K and V gathers
+  // paged KV: one-row boxes for the K and V gathers
   if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : HKEYS) != CUDA_SUCCESS ||
       make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : VKEYS) != CUDA_SUCCESS ||
       make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // output rows as fp32 [rows][512] for the epilogue's 32x32 TMA stores
+  // output rows for the epilogue's TMA stores
   int64_t out_rows = 0;
   for (int b = 0; b < p.B; ++b)
     if (p.T[b] > 0) out_rows = std::max<int64_t>(out_rows, out_row_index(p, b, p.S[b] - 1, p.T[b] * p.H - 1) + 1);
   int o_tma = 0;
   std::memset(&tmap_o, 0, sizeof(tmap_o));
   if (out_rows > 0 && out_rows <= (int64_t)0x7fffffff && (reinterpret_cast<uintptr_t>(a.o) & 15) == 0) {
+    // fp32 [rows][512] in 32x32 boxes, or the fp16 merge partials in 64x32 boxes
     const cuuint64_t dims[2] = {(cuuint64_t)DC, (cuuint64_t)out_rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)DC * 4};
-    const cuuint32_t box[2] = {32, 32};
+    const cuuint64_t strides[1] = {(cuuint64_t)DC * (p.part_f16 ? 2 : 4)};
+    const cuuint32_t box[2] = {p.part_f16 ? 64u : 32u, 32};
     const cuuint32_t estr[2] = {1, 1};
-    o_tma = enc(&tmap_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.o, dims, strides, box, estr,
+    o_tma = enc(&tmap_o, p.part_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.o,
+                dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS ? 1 : 0;
   }

@@ -30,13 +30,14 @@ KDV_DERR_BAD_LENGTH = 3
 KDV_DERR_BAD_TOKEN = 4
 KDV_DERR_TIMEOUT = 5
 KDV_DERR_BAD_SCORE = 6
+KDV_DERR_RANGE = 7
 
 KDV_BF16 = 0
 KDV_F32 = 1
 KDV_IMPL_AUTO = 0
 KDV_IMPL_SIMT = 1
 KDV_IMPL_TC = 2
-KDV_IMPL_TC_1SM = 3
+KDV_IMPL_TC_1SM = 3          # retired: kdv_verify_attn returns KDV_ERR_UNSUPPORTED
 KDV_IMPL_TC_STAGED = 4
 KDV_MAX_TREE = 64
 KDV_MAX_BATCH = 128
@@ -72,7 +73,7 @@ class VerifyParams(ctypes.Structure):
         ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("o_part", ctypes.c_void_p), ("lse_part", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-        ("d_err", ctypes.c_void_p),
+        ("d_err", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64),
     ]
 
 

@@ -1,28 +1,34 @@
 """Parity metric shared by the GPU tests.
 
-Two sets of bars, both checked:
+Bars (the stated tolerance, read on unit-scale outputs): errors of o_lat are
+divided by the RMS of the oracle's o_lat over the tensor, because o_lat
+entries shrink like 1/sqrt(L) with context while the inputs stay N(0,1):
 
-1. The stated tolerance, on absolute errors of o_lat and lse. Every workload
-   draws its activations from N(0,1) (unit scale), so absolute errors are the
-   errors "on unit-scale outputs": max |err| <= 1e-2, mean |err| <= 1e-3,
-   |lse err| <= 1e-3.
+    normalised max |err| <= 1e-2, normalised mean |err| <= 1e-3,
+    |lse err| <= 1e-3 (absolute, natural log).
 
-2. Relative bars, which keep the check sharp at long context where o_lat
-   entries shrink like 1/sqrt(L). Errors are divided by the RMS of the
-   oracle's o_lat. The tensor-core path rounds the softmax numerators P to
-   bf16 before P.V. The unit roundoff is u = 2^-9, so each weight carries a
-   relative error up to u. That alone gives a normalised mean error of about
-   sqrt(2/pi) * u/sqrt(3) ~ 0.9e-3, and a max a few times larger. The bars
-   are mean <= 2e-3 (~2x the bf16 floor) and max <= 3e-2. fp32 paths pass
-   far tighter bars, set per test.
+The absolute errors are held to the same 1e-2 / 1e-3 as well (they are the
+looser pair whenever RMS(o_ref) < 1).
+
+What the bf16 tensor-core path is expected to give: its only rounding beyond
+fp32 accumulation is that of the softmax numerators P, which it rounds to
+fp16 before P.V (unit roundoff 2^-11). Weight j then carries a relative
+error delta_j, uniform within +-2^-11/m_j for mantissa m_j in [1, 2), and
+o's error is sum_j w_j delta_j v_j: normal with standard deviation
+std(delta) * RMS(o), std(delta) = 2^-11 * sqrt(E[1/m^2] / 3) ~ 2.1e-4 for
+log-uniform mantissas. That puts the normalised mean error near
+sqrt(2/pi) * 2.1e-4 ~ 1.7e-4 and the max over ~1e5..1e6 elements at 4-5
+standard deviations, ~1e-3. A CPU emulation of the kernel's arithmetic
+gives 1.3e-4 and 0.6e-3..1.0e-3 on the Kimi-shape cases. fp32 paths pass
+far tighter bars, set per test.
 """
 import numpy as np
 
 MAX_TOL = 1e-2       # absolute, stated
 MEAN_TOL = 1e-3      # absolute, stated
 LSE_TOL = 1e-3       # absolute, stated
-REL_MAX_TOL = 3e-2   # normalised by RMS(o_ref), derived from bf16 P rounding
-REL_MEAN_TOL = 2e-3
+REL_MAX_TOL = 1e-2   # normalised by RMS(o_ref)
+REL_MEAN_TOL = 1e-3
 
 
 def parity_stats(o, lse, o_ref, lse_ref):

@@ -105,15 +105,24 @@ def test_tc_alignment_rejected(lib):
                 q=0x1000, kv=0x2000, kv_off=0x3000, tree_off=0x4000, mask=0x5000, o=0x6000,
                 q_row_stride=577)
     assert lib.kdv_verify_attn(ctypes.byref(p), None) == kdv.KDV_ERR_INVALID_ARG
+    # outputs are written in 16-byte vectors: a 4-byte aligned o is refused
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
+                q=0x1000, kv=0x2000, kv_off=0x3000, tree_off=0x4000, mask=0x5000, o=0x6004)
+    assert lib.kdv_verify_attn(ctypes.byref(p), None) == kdv.KDV_ERR_INVALID_ARG
 
 
 def test_workspace_sizes(lib):
     # forced single split: direct output, no workspace
     assert kdv.kdv_verify_attn_workspace(_params(num_splits=1)) == 0
-    # forced 3 splits, merged by the library: 3 * T*H partial rows of (D_c + 1) floats
+    # forced 3 splits, merged by the library (SIMT kernel): 3 * T*H partial
+    # rows of D_c fp32 values, then one fp32 lse each
     n = kdv.kdv_verify_attn_workspace(_params(num_splits=3))
     parts = 3 * 3 * 4
     assert n == ((parts * 64 * 4 + 255) // 256) * 256 + parts * 4
+    # the tensor-core kernel keeps its merge partials o_k in fp16
+    p = _params(num_splits=3, dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC)
+    n = kdv.kdv_verify_attn_workspace(p)
+    assert n == ((parts * 512 * 2 + 255) // 256) * 256 + parts * 4
     # partials returned to the caller: no workspace
     assert kdv.kdv_verify_attn_workspace(_params(num_splits=3, return_partials=1)) == 0
 

@@ -1,7 +1,6 @@
-"""GPU parity of the tensor-core (tcgen05/TMEM/TMA) verify kernels vs the oracle,
-through the C ABI. Kimi/DeepSeekV3 latent dims (512 + 64), bf16 inputs. Both
-kernels run every case: the 2-SM-MMA kernel (4-CTA clusters, the default) and
-the 1-SM-MMA kernel (2-CTA clusters)."""
+"""GPU parity of the tensor-core (tcgen05/TMEM/TMA) verify kernel vs the oracle,
+through the C ABI. Kimi/DeepSeekV3 latent dims (512 + 64), bf16 inputs, the
+2-SM-MMA kernel on 4-CTA clusters."""
 import math
 
 import numpy as np
@@ -14,9 +13,9 @@ from tests.parity import assert_parity
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_1SM], ids=["tc2sm", "tc1sm"])
-def impl(request):
-    return request.param
+@pytest.fixture
+def impl():
+    return kdv.KDV_IMPL_TC
 
 
 def _run(case, impl, splits=1, partials=False):
@@ -80,8 +79,9 @@ def test_tc_lazy_rescale_growing_logits(impl):
     case = datagen.scaled_case(case, 3.0)
     o, lse = _run(case, impl, splits=1)
     o_ref, lse_ref = oracle.verify_case(case)
-    # inputs here are not unit-scale (|o_lat| ~ 2): only the relative bars apply
-    assert_parity(o, lse, o_ref, lse_ref, max_tol=np.inf, mean_tol=np.inf)
+    # a sharp softmax: the max error is set by the rounding of the few
+    # dominant weights, ~2^-11 * max|v| / RMS(o) ~ 1.5e-3 normalised here
+    assert_parity(o, lse, o_ref, lse_ref)
 
 
 def test_tc_matches_simt_on_same_inputs(impl):
@@ -143,12 +143,6 @@ def test_tc_auto_picks_tc_for_paged():
     np.testing.assert_array_equal(o, o2)
 
 
-def test_tc_1sm_rejects_page_table():
-    case = datagen.make_case("r", **datagen.KIMI, prefix_len=[10], parents=[datagen.chain_tree(2)],
-                             seed=1, paged=True)
-    with pytest.raises(kdv.KdvError) as e:
-        kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_1SM).run()
-    assert e.value.status == kdv.KDV_ERR_UNSUPPORTED
 
 
 # ---------------------------------------------------------------------------

@@ -8,8 +8,7 @@ import pytest
 
 from speculative_tree_verify_mla_b200 import kdv
 
-ROWS_PER_ITEM = {kdv.KDV_IMPL_TC: 256, kdv.KDV_IMPL_TC_STAGED: 256, kdv.KDV_IMPL_TC_1SM: 128,
-                 kdv.KDV_IMPL_SIMT: 8}
+ROWS_PER_ITEM = {kdv.KDV_IMPL_TC: 256, kdv.KDV_IMPL_TC_STAGED: 256, kdv.KDV_IMPL_SIMT: 8}
 
 
 def _plan(L, T, H=64, impl=kdv.KDV_IMPL_AUTO, splits=0, dtype=kdv.KDV_BF16):
@@ -34,10 +33,10 @@ def test_items_are_row_tiles_times_splits(L, T, impl):
     assert items == sum(-(-t * 64 // r) * s for t, s in zip(T, splits))
 
 
-@pytest.mark.parametrize("impl", [kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_1SM])
+@pytest.mark.parametrize("impl", [kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_STAGED])
 @pytest.mark.parametrize("L,T", CASES)
 def test_splits_bounded_by_two_key_tiles_per_split(L, T, impl):
-    """Every split of the tensor-core kernels spans at least two 128-key
+    """Every split of the tensor-core kernel spans at least two 128-key
     tiles (one request's keys n = L + T), so 1 <= S <= ceil(n / 256)."""
     splits, _ = _plan(L, T, impl=impl)
     for l, t, s in zip(L, T, splits):
@@ -61,3 +60,9 @@ def test_splits_never_fall_as_the_prefix_grows():
 def test_plan_rejects_oversized_trees():
     with pytest.raises(RuntimeError):
         _plan([100], [65])
+
+
+def test_retired_one_sm_variant_is_rejected():
+    with pytest.raises(kdv.KdvError) as e:
+        _plan([100], [5], impl=kdv.KDV_IMPL_TC_1SM)
+    assert e.value.status == kdv.KDV_ERR_UNSUPPORTED
