@@ -24,6 +24,17 @@
 #include "sm100_ptx.cuh"
 
 namespace kdv {
+
+// absorb_tc.cu: the tensor-core forms (bf16 weights; see the conditions below)
+size_t absorb_tc_smem(int D_n);
+size_t unabsorb_tc_smem(int D_c);
+cudaError_t launch_absorb_q_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_n,
+                               const void* q_nope, int64_t q_stride, void* q_lat, int64_t o_stride, int32_t o_dtype,
+                               cudaStream_t s);
+cudaError_t launch_unabsorb_o_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_v,
+                                 const float* o_lat, int64_t i_stride, void* out, int64_t o_stride, int32_t o_dtype,
+                                 cudaStream_t s);
+
 namespace {
 
 constexpr int THREADS = 128;
@@ -571,6 +582,15 @@ kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tmap;
+  // tensor cores: bf16 weights and q_nope, whole 128-row weight tiles,
+  // 64-dim K-blocks, 16-byte aligned rows
+  if (vec && q_dtype == KDV_BF16 && d_latent % 128 == 0 && d_nope % 64 == 0 && d_nope <= 256 &&
+      q_nope_stride % 8 == 0 && (reinterpret_cast<uintptr_t>(q_nope) & 15) == 0 &&
+      (int64_t)num_heads * d_latent <= 0x7fffffff &&
+      weight_map(&tmap, w_uk, (uint64_t)num_heads * d_latent, (uint64_t)d_nope, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return launch_absorb_q_tc(tmap, rows, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_lat, q_lat_stride,
+                              out_dtype, s) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
   if (vec && (int64_t)num_heads * d_latent <= 0x7fffffff &&
       weight_map(&tmap, w_uk, (uint64_t)num_heads * d_latent, (uint64_t)d_nope, 64, PA_ROWS,
                  CU_TENSOR_MAP_SWIZZLE_128B)) {
@@ -617,6 +637,14 @@ kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tmap;
+  // tensor cores: bf16 weights, 128-column output tiles, 64-row K-blocks,
+  // 16-byte aligned o_lat rows
+  if (w_dtype == KDV_BF16 && d_v % 128 == 0 && d_latent % 64 == 0 && d_latent <= PU_MAX_DC &&
+      (reinterpret_cast<uintptr_t>(w_uv) & 15) == 0 && (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0 &&
+      o_lat_stride % 4 == 0 && (int64_t)num_heads * d_latent <= 0x7fffffff &&
+      weight_map(&tmap, w_uv, (uint64_t)num_heads * d_latent, (uint64_t)d_v, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return launch_unabsorb_o_tc(tmap, rows, num_heads, d_latent, d_v, o_lat, o_lat_stride, out, out_stride, out_dtype,
+                                s) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
   if (w_dtype == KDV_BF16 && d_v % 8 == 0 && d_latent <= PU_MAX_DC &&
       (reinterpret_cast<uintptr_t>(w_uv) & 15) == 0 && (int64_t)num_heads * d_latent <= 0x7fffffff &&
       weight_map(&tmap, w_uv, (uint64_t)num_heads * d_latent, (uint64_t)d_v, PU_V, 256,

@@ -107,11 +107,14 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + QK_BLOCKS * QBLOCK_BYTES;
 constexpr int OFF_XCHG = OFF_KV + KV_STAGES * KBLOCK_BYTES;   // float [2][2][128] + [128] (S side)
 constexpr int XCHG_BYTES = 5 * ROWS * 4;
+constexpr int OFF_KSLOT = OFF_XCHG + XCHG_BYTES;             // int32 [128] (S side, paged KV)
 constexpr int OFF_VRING = 0;
 constexpr int OFF_P = OFF_VRING + V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
 constexpr int OFF_VSLOT = OFF_STATS + STATS_BYTES;            // int32 [256] (O side, paged KV)
-constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
+constexpr int EPI_STAGE_BYTES = 16384;                         // per epilogue warp, over V ring + P slots
+static_assert(OFF_VRING + 8 * EPI_STAGE_BYTES <= OFF_STATS, "epilogue staging overlaps the row statistics");
+constexpr int OFF_MISC = OFF_KSLOT + HKEYS * 4;
 static_assert(OFF_VSLOT + STILE * 4 <= OFF_MISC, "O-side buffers overlap misc");
 constexpr int OFF_BAR = OFF_MISC;
 constexpr int NUM_BARS = 56;
@@ -203,12 +206,15 @@ __device__ __forceinline__ bool wait_warp(const Ctx& c, uint32_t bar, uint32_t p
 }
 
 // Arrive on barrier `bar` (local offset) of CTA `rank`: a local arrive when
-// it is this CTA, else a relaxed remote arrive. No cross-CTA arrival here
-// publishes generic-proxy data: each follows tcgen05.ld / tcgen05.st work the
-// thread has already waited for (tcgen05.wait) or guards bytes that reach the
-// other side through complete_tx. A release-ordered remote arrive costs
-// ~1800 cycles on this part against ~440 for a relaxed one (measured), enough
-// to starve the pipeline.
+// it is this CTA, else a relaxed remote arrive. Every cross-CTA arrival in
+// this kernel is relaxed. Each follows work the arriving thread has already
+// completed -- tcgen05.ld / tcgen05.st it waited for (tcgen05.wait), bytes
+// that reached its CTA through complete_tx, or its own shared-memory stores
+// of a V stage -- and, where the pair's MMA will read shared memory of the
+// arriving CTA, a fence.proxy.async that orders that CTA's writes before
+// async-proxy reads. A release-ordered remote arrive costs ~1800 cycles on
+// this part against ~440 for a relaxed one (measured), enough to starve the
+// pipeline.
 __device__ __forceinline__ void arrive_on(uint32_t bar, uint32_t rank, uint32_t my_rank) {
   if (rank == my_rank) mbar_arrive(bar);
   else mbar_arrive_remote_relaxed(mapa(bar, rank));
@@ -273,7 +279,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
     reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR)[0] = 0;
     if (s_side) {
       for (int i = 0; i < KV_STAGES; ++i) {
-        mbar_init(c.bar(B_KV_FULL + i), 1);
+        // TMA: the leader's expect_tx arrival (bytes of both CTAs counted);
+        // paged cp.async: one arrival from each CTA's producer
+        mbar_init(c.bar(B_KV_FULL + i), PAGED ? 2 : 1);
         mbar_init(c.bar(B_KV_EMPTY + i), 1);
       }
       for (int i = 0; i < 2; ++i) {
@@ -289,7 +297,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       for (int i = 0; i < V_STAGES; ++i) {
         mbar_init(c.bar(B_V_FULL + i), 2 * CONVERTERS);   // the converter warps of both O CTAs
         mbar_init(c.bar(B_V_EMPTY + i), 1);
-        mbar_init(c.bar(B_V_LANDED + i), 1);
+        mbar_init(c.bar(B_V_LANDED + i), PAGED ? 32 : 1);   // TMA bytes, or each producer lane's copies
       }
       for (int i = 0; i < NP; ++i) {
         mbar_init(c.bar(B_P_FULL + i), 1);
@@ -326,14 +334,26 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // ---------------- producer (both S CTAs): this CTA's 128 query rows
       // (nine K-blocks, kept for the whole item) and its 128 of every 256 KV
       // rows, one K-block per ring stage; everything counts on the leader's
-      // barriers. Contiguous KV: the next tile's rows are prefetched into L2
-      // while this tile streams. Paged KV: the whole warp gathers, 4 rows per
-      // lane.
+      // barriers. Contiguous KV: TMA boxes, and the next tile's rows are
+      // prefetched into L2 while this tile streams. Paged KV: the whole warp
+      // copies each stage with 16-byte cp.async (eight lanes per pool row,
+      // four rows per instruction) into the same swizzled layout, retires it
+      // three stages later (cp.async.wait_group), orders it for the tensor
+      // core's async-proxy reads and tells the leader with one arrival.
       const int n_stg = n_stiles * QK_BLOCKS;
       int issued = 0;
-      // paged KV: lane l gathers keys 4l..4l+3 of this CTA's 128; their slots
-      // are read one tile ahead so the page-table latency stays off the path
-      int32_t slot[4] = {0, 0, 0, 0}, nslot[4] = {0, 0, 0, 0};
+      // paged KV: lane l looks up keys 4l..4l+3 of this CTA's 128 one tile
+      // ahead (so the page-table latency stays off the path) and publishes
+      // them in a shared table when the tile starts
+      int32_t nslot[4] = {0, 0, 0, 0};
+      int32_t* kslot = reinterpret_cast<int32_t*>(smem + OFF_KSLOT);
+      const char* kv_bytes = static_cast<const char*>(a.kv);
+      // paged KV: stage g's copies are retired and announced to the leader
+      auto announce = [&](int g) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) arrive_on(c.bar(B_KV_FULL + g % KV_STAGES), lead_rank, rank);
+      };
       if (PAGED && n_stiles > 0) {
         const int j0 = stile_key(0) + (int)half * HKEYS + 4 * lane;
 #pragma unroll
@@ -347,27 +367,44 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
                            blk * 64, qy);
         }
       }
+      // A free ring stage is waited for like a drain (no abort check, 1 s):
+      // both producers of the pair watch the same multicast commits, so they
+      // issue the same stages -- the leader's drain below covers the pair's
+      // loads only if neither producer goes on after the other stopped.
       for (int g = 0; g < n_stg; ++g) {
         const int st = g % KV_STAGES;
         const uint32_t eparity = ((g / KV_STAGES) & 1) ^ 1;
-        if (!(PAGED ? wait_warp(c, c.bar(B_KV_EMPTY + st), eparity) : wait_bar(c, c.bar(B_KV_EMPTY + st), eparity)))
+        if (!(PAGED ? wait_warp(c, c.bar(B_KV_EMPTY + st), eparity, true)
+                    : wait_bar(c, c.bar(B_KV_EMPTY + st), eparity, true)))
           break;
-        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
         const int tile = g / QK_BLOCKS, blk = g % QK_BLOCKS;
-        const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
         const uint32_t dst = base + OFF_KV + st * KBLOCK_BYTES;
         if (PAGED) {
           if (blk == 0) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) slot[q] = nslot[q];
+            for (int q = 0; q < 4; ++q) kslot[4 * lane + q] = nslot[q];
+            __syncwarp();
             if (tile + 1 < n_stiles) {
               const int j0 = stile_key(tile + 1) + (int)half * HKEYS + 4 * lane;
 #pragma unroll
               for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
             }
           }
-          tma_gather4_pair(dst + lane * 512, &tmap_kv, fb, blk * 64, slot[0], slot[1], slot[2], slot[3]);
+          const int ch = lane & 7;
+#pragma unroll 4
+          for (int i = 0; i < HKEYS / 4; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            cp_async16(dst + r * 128 + ((ch ^ (r & 7)) << 4),
+                       kv_bytes + (int64_t)kslot[r] * (DQ * 2) + blk * 128 + ch * 16);
+          }
+          cp_async_commit();
+          if (g >= KV_STAGES - 1) {
+            cp_async_wait<KV_STAGES - 1>();
+            announce(g - (KV_STAGES - 1));
+          }
         } else {
+          if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
+          const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
           const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
           if (blk == 0 && tile + 1 < n_stiles)
             for (int e = 0; e < QK_BLOCKS; ++e) tma_prefetch_l2(&tmap_kv, e * 64, y + STILE);
@@ -375,12 +412,18 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         }
         issued = g + 1;
       }
+      if (PAGED) {
+        // retire this CTA's own copies; announce the stages not yet announced
+        cp_async_wait<0>();
+        for (int g = max(0, issued - (KV_STAGES - 1)); g < issued; ++g) announce(g);
+      }
       if (leader && lane == 0) {
-        // retire copies in flight (both halves count on the leader's barriers)
+        // retire copies in flight (TMA: both halves count on the leader's barriers)
         if (n_stiles > 0)
           for (int blk = 0; blk < QK_BLOCKS; ++blk) wait_bar(c, c.bar(B_Q_FULL + blk), 0, true);
-        for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
-          wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
+        if (!PAGED)
+          for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
+            wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
       }
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T,
@@ -550,7 +593,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // ---------------- V producer (both O CTAs): this CTA's 256 dims of
       // every 32 keys, landing on this CTA's own V_LANDED barrier; local
       // block lb holds dims 64*((lb/2)*4 + half*2 + lb%2), bf16, 128B-swizzled.
-      // Paged KV: lanes 0-7 gather 4 rows each.
+      // Paged KV: the whole warp copies with 16-byte cp.async, one key's four
+      // 128-byte blocks per instruction, and each lane's copies arrive on
+      // V_LANDED when they complete.
       int issued = 0;
       const int n_sub = (STILE / VKEYS) * n_stiles;
       // paged KV: the 256 slots of an S tile sit in a shared table (lane l
@@ -564,10 +609,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
         const uint32_t eparity = ((u / V_STAGES) & 1) ^ 1;
-        if (!(PAGED ? wait_warp(c, c.bar(B_V_EMPTY + st), eparity) : wait_bar(c, c.bar(B_V_EMPTY + st), eparity)))
+        if (!(PAGED ? wait_warp(c, c.bar(B_V_EMPTY + st), eparity, true)
+                    : wait_bar(c, c.bar(B_V_EMPTY + st), eparity, true)))
           break;
         const uint32_t lb_bar = c.bar(B_V_LANDED + st);
-        if (lane == 0) mbar_arrive_expect_tx(lb_bar, V_STAGE_BYTES);
+        if (!PAGED && lane == 0) mbar_arrive_expect_tx(lb_bar, V_STAGE_BYTES);
         const int key0 = stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS;
         const uint32_t dst = base + OFF_VRING + st * V_STAGE_BYTES;
         if (PAGED) {
@@ -581,18 +627,15 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             }
             __syncwarp();
           }
-          if (lane < VKEYS / 4) {
-            const int k = key0 - stile_key(vt) + 4 * lane;
-            int32_t slot[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) slot[q] = vslot[k + q];
-            for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
-              const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-              tma_gather4(dst + lb * VBLOCK_BYTES + lane * 512, &tmap_v, lb_bar, gb * 64, slot[0], slot[1], slot[2],
-                          slot[3]);
-            }
-          }
-          __syncwarp();
+          const int lb = lane >> 3, ch = lane & 7;
+          const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
+          const char* src0 = static_cast<const char*>(a.kv) + gb * 128 + ch * 16;
+          const int k0 = key0 - stile_key(vt);
+#pragma unroll 4
+          for (int k = 0; k < VKEYS; ++k)
+            cp_async16(dst + lb * VBLOCK_BYTES + k * 128 + ((ch ^ (k & 7)) << 4),
+                       src0 + (int64_t)vslot[k0 + k] * (DQ * 2));
+          cp_async_arrive_noinc(lb_bar);
         } else {
           const int32_t y = (int32_t)(kv_base + key0);
           for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
@@ -741,12 +784,15 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             }
             st_shared_v4(addr, v.x, v.y, v.z, v.w);
           }
-          // the pair's MMA reads these bytes through the async proxy
+          // the pair's MMA reads these bytes through the async proxy: every
+          // thread orders its stores before async-proxy reads, then one
+          // relaxed arrive per warp (as for the P tiles; a release-ordered
+          // remote arrive would stall the warp ~1800 cycles per stage)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             if (leader) mbar_arrive(c.bar(B_V_FULL + st));
-            else mbar_arrive_remote(vfull_lead + st * 8);
+            else mbar_arrive_remote_relaxed(vfull_lead + st * 8);
           }
         }
         if (__any_sync(0xffffffffu, range != 0) && lane == 0) record_error(a.d_err, KDV_DERR_RANGE);
@@ -762,14 +808,15 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const float lse = (l > 0.f && !bad) ? (m + __log2f(l)) * LN2 : -INFINITY;
       const int64_t orow = out_row_index(p, b, split, row);
       // Whole-warp rows go out through TMA stores of 4 KB boxes staged
-      // 128B-swizzled in the V ring (free once the last PV is done): 32 rows
-      // x 32 fp32 columns, or, for the internal merge's fp16 partials, 32
-      // rows x 64 fp16 columns. A warp straddling the end of the request
-      // stores row by row.
+      // 128B-swizzled in the V ring and P slots (free once the last PV is
+      // done; 16 KB per warp, four boxes in flight): 32 rows x 32 fp32
+      // columns, or, for the internal merge's fp16 partials, 32 rows x 64
+      // fp16 columns. A warp straddling the end of the request stores row by
+      // row.
       const int wrow0 = row0 + sp * 32;
       const bool warp_full = o_tma != 0 && !bad && wrow0 + 32 <= rows_b;
       const int64_t wy = out_row_index(p, b, split, wrow0);
-      const uint32_t stage = base + OFF_VRING + ew * 8192;
+      const uint32_t stage = base + OFF_VRING + ew * EPI_STAGE_BYTES;
       const int cols_per_box = p.part_f16 ? 64 : 32;
 #pragma unroll 1
       for (int cb = 0; cb < 256 / cols_per_box; ++cb) {
@@ -803,9 +850,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * inv);
         }
         if (warp_full) {
-          const uint32_t buf = stage + (cb & 1) * 4096;
-          if (cb >= 2) {
-            if (lane == 0) bulk_wait_group_read<1>();
+          const uint32_t buf = stage + (cb & 3) * 4096;
+          if (cb >= 4) {
+            if (lane == 0) bulk_wait_group_read<3>();
             __syncwarp();
           }
 #pragma unroll
