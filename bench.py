@@ -126,7 +126,8 @@ def tensor_fracs(tflops: float, peaks) -> dict:
             "peak_datasheet": DATASHEET_PEAKS["bf16_tflops"]}
 
 
-TC_KERNEL = {2: ("verify_tc2_kernel", "verify_tc2.cu"), 4: ("verify_tc2_kernel", "verify_tc2.cu")}
+TC_KERNEL = {0: ("verify_tc2_kernel", "verify_tc2.cu"), 2: ("verify_tc2_kernel", "verify_tc2.cu"),
+             4: ("verify_tc2_kernel", "verify_tc2.cu")}
 
 
 def kernel_source_hash(src="verify_tc2.cu"):
@@ -283,7 +284,8 @@ class Problems:
     """The step's verify problems, resident on the device: one kdv_verify_attn
     call per case (inputs, outputs, workspace), masks shared by cases whose
     trees are identical, and a partials-out twin of every call for timing the
-    tensor-core kernel alone."""
+    tensor-core kernel alone (given its fp16 latent rows, prepared once, so
+    that the twin launches only the attention kernel)."""
 
     def __init__(self, cases, impl_code, dev):
         import torch
@@ -295,6 +297,8 @@ class Problems:
         self.q, self.kv, self.o, self.lse, self.ws, self.params, self.tc_params = [], [], [], [], [], [], []
         self.page_table, self.kv_off, self.tree_off, self.keep = [], [], [], []
         self.splits, self.items, self.n_combine = [], [], 0
+        self.v16, self.n_keys = [], []
+        self.tc = impl_code in (kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_STAGED, kdv.KDV_IMPL_AUTO)
         for c in cases:
             key = c.parent.tobytes() + c.tree_off.tobytes()
             if key not in self.trees:
@@ -328,6 +332,12 @@ class Problems:
             tp = kdv.make_params(**common, num_splits=S, return_partials=1, o=None, lse=None,
                                  o_part=o_part, lse_part=lse_part, workspace=None,
                                  workspace_bytes=0)
+            n_keys = int((c.prefix_len + c.tree_T).sum())
+            v16 = torch.empty(n_keys, 512, dtype=torch.float16, device=dev)
+            kdv.kdv_latent_f16(tp, v16)
+            tp.v16 = v16.data_ptr()
+            self.v16.append(v16)
+            self.n_keys.append(n_keys)
             tbytes = kdv.kdv_verify_attn_workspace(tp)       # staged paged rows, if any
             tws = torch.empty(max(16, tbytes), dtype=torch.uint8, device=dev)
             tp.workspace, tp.workspace_bytes = tws.data_ptr(), tbytes
@@ -349,8 +359,16 @@ class Problems:
         for p in self.tc_params:
             kdv.kdv_verify_attn(p, s)
 
+    def latent_only(self, s):
+        """The fp16 latent-row pass of every call alone."""
+        from speculative_tree_verify_mla_b200 import kdv
+        for p, v in zip(self.tc_params, self.v16):
+            kdv.kdv_latent_f16(p, v, s)
+
     def launches_per_step(self):
-        return len(self.trees) + len(self.params) + self.n_combine
+        # mask builds, then per call: the fp16 latent rows, the attention
+        # kernel and (with splits) the merge
+        return len(self.trees) + (2 if self.tc else 1) * len(self.params) + self.n_combine
 
 
 def graph_of(fn, stream):
@@ -485,7 +503,7 @@ def time_tree_build(dev, stream, budget: int = 32, n_calls: int = 64, reps: int 
     return res
 
 
-def time_config(name: str, dev, stream, peaks, impl_code: int = 2, reps: int = 20):
+def time_config(name: str, dev, stream, peaks, impl_code: int = 0, reps: int = 20):
     """One of the other verify configurations as a sub-record of the headline
     line: the whole kdv_verify_attn call (kernel + split merge) and the
     tensor-core kernel alone (the partials-out twin, same grid), each from a
@@ -543,6 +561,7 @@ def run_gpu(args):
     stream.synchronize()
     g_step = graph_of(prob.step, stream)
     g_tc = graph_of(prob.tc_only, stream)
+    g_lat = graph_of(prob.latent_only, stream)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(dev.index if world == 1 else local)
@@ -569,6 +588,7 @@ def run_gpu(args):
 
     # dominant kernel alone (same grid, partials out): per-launch duration
     tc_us = replay_us(g_tc, stream, max(3, min(50, args.steps // 4))) / len(prob.params)
+    lat_us = replay_us(g_lat, stream, max(3, min(50, args.steps // 4))) / len(prob.params)
     clocks = sampler.stop()
     assert int(prob.d_err.item()) == 0, f"device error flag {int(prob.d_err.item())}"
 
@@ -668,8 +688,18 @@ def run_gpu(args):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tc_tflops / peaks["bf16_tflops"], "traffic": traffic,
                      "us_per_launch": tc_us, "flops_per_launch": flops,
-                     "kv_bytes_per_launch": kv_bytes, "peak_source": peaks["source"] + " burst bf16",
+                     "kv_bytes_per_launch": kv_bytes,
+                     # what the kernel itself must read: the bf16 rows (its QK^T), the fp16
+                     # latent rows (its P.V) and the query rows -- compare with traffic
+                     "read_bytes_per_launch": kv_bytes + prob.n_keys[0] * 1024.0 + c0.rows * 1152.0,
+                     "peak_source": peaks["source"] + " burst bf16",
                      **tensor_fracs(tc_tflops, peaks)},
+        "latent_f16": {"kernel": "latent_f16_kernel", "us_per_call": lat_us, "bound": "hbm",
+                       "bytes_per_call": prob.n_keys[0] * 2048.0,
+                       "achieved_gbs": prob.n_keys[0] * 2048.0 / (lat_us * 1e-6) / 1e9,
+                       "frac": prob.n_keys[0] * 2048.0 / (lat_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                       "note": "bf16 c_kv -> fp16 rows read by the attention kernel's P.V; "
+                               "1 KB read + 1 KB written per key; included in value"},
         "e2e": {"value": e2e_ms * 1e3 / n_calls, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": args.steps * prob.launches_per_step(),
@@ -703,7 +733,7 @@ def run_gpu(args):
     if rank == 0:
         print(json.dumps(result))
     if world > 1:
-        del g_step, g_tc
+        del g_step, g_tc, g_lat
         torch.distributed.destroy_process_group()
     return 0
 
@@ -716,9 +746,10 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT)
     ap.add_argument("--impl", choices=["kdv", "reference"], default="kdv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["tc2", "tc2s"], default="tc2",
-                    help="tensor-core kernel: 2-SM MMAs (default), or the same over a staged "
-                         "contiguous copy of a paged pool")
+    ap.add_argument("--kernel", choices=["auto", "tc2", "tc2s"], default="auto",
+                    help="auto (default: what KDV_IMPL_AUTO picks -- the tensor-core kernel, over a "
+                         "staged contiguous copy when the pool is paged), tc2 (the tensor-core "
+                         "kernel, gathering a paged pool through its page table), tc2s (staged)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kimi",
                     help="kimi (default, the headline): " + WORKLOADS["kimi"] + "; sweep: "
                          + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
@@ -727,7 +758,7 @@ def parse_args(argv=None):
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the sub-records (other configurations, acceptance, projections, builder)")
     args = ap.parse_args(argv)
-    args.impl_code = {"tc2": 2, "tc2s": 4}[args.kernel]
+    args.impl_code = {"auto": 0, "tc2": 2, "tc2s": 4}[args.kernel]
     args.warmup = max(3, args.warmup)
     return args
 

@@ -79,25 +79,27 @@ typedef enum {
 #define KDV_F32 1
 
 /* Kernel family for kdv_verify_attn. AUTO picks the tensor-core kernel when
- * its shape constraints hold (bf16, d_latent=512, d_rope=64), else SIMT. TC
- * runs 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per work item):
- * Q.K^T in bf16, P.V with P and V in fp16 (11 significant bits, so the
- * rounding of the softmax numerators costs ~1.3e-4 of the output's RMS
- * instead of ~1e-3 in bf16). The c_kv values it reads must therefore lie in
- * fp16's range, |x| < 65536 (KDV_DERR_RANGE otherwise); rows past a
- * request's last key are never read. A paged pool is read with TMA four-row
- * gathers (keys) and per-row loads (values). Value 3 (a 1-SM-MMA variant of
- * earlier versions) is retired and returns KDV_ERR_UNSUPPORTED. */
+ * its shape constraints hold (bf16, d_latent=512, d_rope=64) -- through a
+ * staged copy (TC_STAGED) when there is a page table -- else SIMT. TC runs
+ * 2-SM tcgen05 MMAs on 4-CTA clusters (256 query rows per work item): Q.K^T
+ * in bf16, P.V with P and V in fp16 (11 significant bits, so the rounding of
+ * the softmax numerators costs ~1.5e-4 of the output's RMS instead of ~1e-3
+ * in bf16). V is read from fp16 rows that the call writes first (see
+ * kdv_latent_f16), so the c_kv values it reads must lie in fp16's range,
+ * |x| < 65536 (KDV_DERR_RANGE otherwise); pool rows outside the requests'
+ * keys are never read for P.V. TC reads a paged pool's keys in place with
+ * TMA four-row gathers. Value 3 (a 1-SM-MMA variant of earlier versions) is
+ * retired and returns KDV_ERR_UNSUPPORTED. */
 #define KDV_IMPL_AUTO 0
 #define KDV_IMPL_SIMT 1
 #define KDV_IMPL_TC 2
 #define KDV_IMPL_TC_1SM 3
 /* TC_STAGED: the 2-SM kernel over a paged pool, first copying every request's
- * rows (in logical order) into a contiguous region of the workspace and then
- * reading them with tiled TMA boxes instead of four-row gathers. Faster for
- * paged pools (about 2x on the 8-request batched workload) at the price of
- * workspace = (sum of L_b + T_b) x (D_c + D_r) x 2 bytes more. Without a page
- * table it is KDV_IMPL_TC. */
+ * rows (in logical order) into a contiguous region of the workspace -- in the
+ * same pass that writes the fp16 rows -- and then reading them with tiled
+ * TMA boxes instead of four-row gathers. Faster for paged pools at the price
+ * of workspace = (sum of L_b + T_b) x (D_c + D_r) x 2 bytes more; AUTO's
+ * choice for paged pools. Without a page table it is KDV_IMPL_TC. */
 #define KDV_IMPL_TC_STAGED 4
 
 #define KDV_MAX_TREE 64    /* nodes per tree (one 64-bit mask word)          */
@@ -108,7 +110,9 @@ KDV_API const char* kdv_status_string(kdv_status s);
 
 /* Library ABI version (major*100 + minor): 110 adds kdv_tree_accept,
  * kdv_tree_build, kdv_absorb_q / kdv_unabsorb_o and KDV_IMPL_TC_STAGED to
- * the 100 set (mask build, verify, no-alloc verify, combine). */
+ * the 100 set (mask build, verify, no-alloc verify, combine); 120 adds
+ * kdv_latent_f16, the wait_limit_ns and v16 fields of kdv_verify_params,
+ * KDV_DERR_RANGE, and retires KDV_IMPL_TC_1SM. */
 KDV_API int32_t kdv_version(void);
 
 /*
@@ -179,10 +183,18 @@ typedef struct kdv_verify_params {
                               its copies and MMAs in flight (waiting up to 1 s
                               for them) and exits normally, its outputs not
                               valid. A small value is for testing that path. */
+  const void* v16;       /* TC kernel, nullable: the fp16 latent rows of this
+                            call, as kdv_latent_f16 writes them for these
+                            parameters (a caller that mirrors its latent cache
+                            in fp16 keeps them up to date and saves the
+                            conversion); NULL = the call writes them into its
+                            workspace before the attention kernel runs        */
 } kdv_verify_params;
 
 /* Bytes of workspace kdv_verify_attn needs for these parameters (the plan
- * depends only on the host fields). Writes *bytes; may be 0. */
+ * depends only on the host fields). Writes *bytes; may be 0. For the TC
+ * kernel it includes the fp16 latent rows (sum_b (L_b + T_b) x 1 KB) unless
+ * p->v16 is given. */
 KDV_API kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t* bytes);
 
 /* The plan kdv_verify_attn would use for these parameters (host fields only):
@@ -203,6 +215,23 @@ KDV_API kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* spl
  * multiples of 16 bytes (KDV_ERR_INVALID_ARG otherwise).
  */
 KDV_API kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream);
+
+/*
+ * kdv_latent_f16 -- the fp16 copy of the latent rows that the tensor-core
+ * kernel's P.V reads (this library's design, not the pages': its P.V runs
+ * in fp16, whose 11 significant bits keep the rounding of the softmax
+ * numerators ~8x below bf16's, and an MMA needs both operands in one type).
+ * Writes the c_kv part (D_c = 512 dims) of every key the call reads --
+ * request b's logical keys j = 0 .. L_b+T_b-1, through the page table when
+ * there is one -- as fp16 to row sum_{b'<b}(L_b'+T_b') + j of
+ * v16 [sum_b (L_b+T_b)][512] (device, 16-byte aligned). bf16 -> fp16 is
+ * exact for 2^-14 <= |x| < 65536; smaller values round to subnormals.
+ * Device errors: KDV_DERR_RANGE (|x| >= 65536, inf or NaN in a row it
+ * reads), KDV_DERR_BAD_SLOT / KDV_DERR_BAD_LENGTH (a row outside the pool;
+ * written as zeros). kdv_verify_attn calls it itself unless p->v16 is set.
+ * Requires the TC shape (bf16, d_latent 512, d_rope 64); p->impl is ignored.
+ */
+KDV_API kdv_status kdv_latent_f16(const kdv_verify_params* p, void* v16, void* stream);
 
 /*
  * kdv_verify_attn_noalloc -- kdv_verify_attn for callers that cannot allocate.

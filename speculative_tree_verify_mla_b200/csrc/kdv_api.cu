@@ -8,12 +8,6 @@
 
 #include "kdv_internal.cuh"
 
-namespace kdv {
-// stage_kv.cu: copy the paged rows of every request to contiguous staged rows
-cudaError_t launch_stage_kv(const VerifyArgs& a, const VerifyPlan& p, int32_t row_bytes, void* staged,
-                            int32_t* staged_off, cudaStream_t stream);
-}  // namespace kdv
-
 using namespace kdv;
 
 namespace {
@@ -38,9 +32,13 @@ bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED;
 // the 2-SM kernel, reading the pool directly or a staged copy
 bool is_tc2(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED; }
 
+// AUTO: the tensor-core kernel when its shape constraints hold, reading a
+// paged pool through a staged contiguous copy (the fastest path, at the
+// price of workspace for the copy); else SIMT.
 int resolve_impl(const kdv_verify_params* p) {
   if (p->impl == KDV_IMPL_SIMT || is_tc(p->impl)) return p->impl;
-  return tc_shape_ok(p) ? KDV_IMPL_TC : KDV_IMPL_SIMT;
+  if (!tc_shape_ok(p)) return KDV_IMPL_SIMT;
+  return p->page_table != nullptr ? KDV_IMPL_TC_STAGED : KDV_IMPL_TC;
 }
 
 // Host-side checks that need no device access.
@@ -91,6 +89,7 @@ kdv_status check_pointers(const kdv_verify_params* p, int impl) {
     if (!aligned16(p->q) || !aligned16(p->kv)) return KDV_ERR_INVALID_ARG;
     if ((stride * (int64_t)esz) % 16 != 0) return KDV_ERR_INVALID_ARG;
     if ((p->o && !aligned16(p->o)) || (p->o_part && !aligned16(p->o_part))) return KDV_ERR_INVALID_ARG;
+    if (p->v16 && !aligned16(p->v16)) return KDV_ERR_INVALID_ARG;
   }
   float* outs[4] = {p->o, p->lse, p->o_part, p->lse_part};
   for (float* f : outs)
@@ -111,6 +110,18 @@ size_t merge_o_bytes(const VerifyPlan& plan, int32_t d) {
 size_t merge_region_bytes(const VerifyPlan& plan, int32_t d) {
   return merge_o_bytes(plan, d) + plan_parts(plan) * sizeof(float);
 }
+// Keys a call reads, over all requests.
+int64_t plan_keys(const VerifyPlan& plan) {
+  int64_t n = 0;
+  for (int b = 0; b < plan.B; ++b) n += (int64_t)plan.L[b] + plan.T[b];
+  return n;
+}
+// Workspace layout: [merge partials (OUT_WORKSPACE)] [fp16 latent rows (TC)]
+// [staged rows (TC_STAGED with a page table)], each region 256-byte aligned.
+size_t v16_offset(const VerifyPlan& plan, int32_t d) {
+  return plan.out_mode == OUT_WORKSPACE ? align256(merge_region_bytes(plan, d)) : 0;
+}
+size_t v16_bytes(const VerifyPlan& plan) { return (size_t)plan_keys(plan) * 512 * 2; }
 
 // KDV_IMPL_TC_STAGED with a page table: the pool rows are first copied to a
 // contiguous staged region of the workspace.
@@ -218,6 +229,12 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   }
   plan->item_base[B] = (int32_t)items;
   plan->n_items = (int32_t)items;
+  int64_t v16_rows = 0;
+  for (int b = 0; b < B; ++b) {
+    plan->v16_base[b] = (int32_t)v16_rows;
+    v16_rows += (int64_t)plan->L[b] + plan->T[b];
+    if (v16_rows > INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
+  }
   *ws_bytes = 0;
   if (p->return_partials) {
     plan->out_mode = OUT_PARTIALS;
@@ -231,11 +248,10 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
     plan->part_f16 = is_tc2(impl) ? 1 : 0;
     *ws_bytes = merge_region_bytes(*plan, p->d_latent);
   }
+  if (is_tc2(impl) && p->v16 == nullptr) *ws_bytes = v16_offset(*plan, p->d_latent) + align256(v16_bytes(*plan));
   if (staged_paged(p, impl)) {
-    // after the merge region: staged row offsets [B+1], then the staged rows
-    size_t n_keys = 0;
-    for (int b = 0; b < B; ++b) n_keys += (size_t)plan->L[b] + plan->T[b];
-    if (n_keys > (size_t)INT_MAX / 2) return KDV_ERR_UNSUPPORTED;
+    // after the fp16 rows: staged row offsets [B+1], then the staged rows
+    const size_t n_keys = (size_t)plan_keys(*plan);
     *ws_bytes = align256(*ws_bytes) + align256((size_t)(B + 1) * sizeof(int32_t)) +
                 n_keys * (size_t)(p->d_latent + p->d_rope) * 2;
   }
@@ -259,7 +275,7 @@ const char* kdv_status_string(kdv_status s) {
   return "KDV_ERR_UNKNOWN";
 }
 
-int32_t kdv_version(void) { return 110; }
+int32_t kdv_version(void) { return 120; }
 
 kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
                                int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
@@ -342,25 +358,61 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.lse = ws_l;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // One pass over the pool rows the call reads: the fp16 latent rows of the
+  // P.V operand (unless the caller gave them) and, for a staged paged pool,
+  // the contiguous bf16 copy the kernel then reads with tiled boxes.
+  const void* v16 = p->v16;
+  void* own_v16 = nullptr;
+  void* staged = nullptr;
+  int32_t* staged_off = nullptr;
+  if (is_tc2(impl) && v16 == nullptr) {
+    own_v16 = static_cast<char*>(p->workspace) + v16_offset(plan, p->d_latent);
+    v16 = own_v16;
+  }
   if (staged_paged(p, impl)) {
-    const size_t merge_bytes = plan.out_mode == OUT_WORKSPACE ? merge_region_bytes(plan, p->d_latent) : 0;
-    char* region = static_cast<char*>(p->workspace) + align256(merge_bytes);
-    int32_t* staged_off = reinterpret_cast<int32_t*>(region);
-    void* staged = region + align256((size_t)(plan.B + 1) * sizeof(int32_t));
-    int64_t n_keys = 0;
-    for (int b = 0; b < plan.B; ++b) n_keys += (int64_t)plan.L[b] + plan.T[b];
-    cudaError_t e0 = launch_stage_kv(a, plan, (p->d_latent + p->d_rope) * 2, staged, staged_off, s);
-    if (e0 != cudaSuccess) return KDV_ERR_CUDA;
+    char* region = static_cast<char*>(p->workspace) + v16_offset(plan, p->d_latent) +
+                   (p->v16 == nullptr ? align256(v16_bytes(plan)) : 0);
+    staged_off = reinterpret_cast<int32_t*>(region);
+    staged = region + align256((size_t)(plan.B + 1) * sizeof(int32_t));
+  }
+  if (own_v16 != nullptr || staged != nullptr) {
+    if (launch_latent_f16(a, plan, own_v16, staged, staged_off, s) != cudaSuccess) return KDV_ERR_CUDA;
+  }
+  if (staged != nullptr) {
     a.kv = staged;
-    a.num_slots = n_keys;
+    a.num_slots = plan_keys(plan);
     a.page_table = nullptr;
     a.kv_off = staged_off;
   }
-  cudaError_t e = is_tc2(impl) ? launch_verify_tc2(a, plan, s) : launch_verify_simt(a, plan, p->dtype, s);
+  cudaError_t e = is_tc2(impl) ? launch_verify_tc2(a, plan, v16, plan_keys(plan), s)
+                               : launch_verify_simt(a, plan, p->dtype, s);
   if (e != cudaSuccess) return KDV_ERR_CUDA;
   if (plan.out_mode == OUT_WORKSPACE)
     e = launch_combine_plan(ws_o, ws_l, plan, p->d_latent, p->o, p->lse, s);
   return cuda_status(e);
+}
+
+kdv_status kdv_latent_f16(const kdv_verify_params* p, void* v16, void* stream) {
+  if (p == nullptr || v16 == nullptr || !aligned16(v16)) return KDV_ERR_INVALID_ARG;
+  kdv_verify_params q = *p;
+  q.impl = KDV_IMPL_TC;
+  kdv_status st = check_params(&q, KDV_IMPL_TC);
+  if (st != KDV_OK) return st;
+  if (!q.kv || !q.kv_off || !aligned16(q.kv) || q.num_slots < 0) return KDV_ERR_INVALID_ARG;
+  VerifyPlan plan;
+  size_t need = 0;
+  st = make_plan(&q, KDV_IMPL_TC, &plan, &need);
+  if (st != KDV_OK) return st;
+  VerifyArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kv = q.kv;
+  a.num_slots = q.num_slots;
+  a.page_table = q.page_table;
+  a.kv_off = q.kv_off;
+  a.D_c = q.d_latent;
+  a.D_r = q.d_rope;
+  a.d_err = q.d_err;
+  return cuda_status(launch_latent_f16(a, plan, v16, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
 kdv_status kdv_combine(const float* o_part, const float* lse_part, int32_t S, int64_t rows,

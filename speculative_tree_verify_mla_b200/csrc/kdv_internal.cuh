@@ -29,6 +29,7 @@ struct VerifyPlan {
   int32_t tiles[KDV_MAX_BATCH];
   int32_t tree_base[KDV_MAX_BATCH];   // tree_off[b] (from the host T copies)
   int32_t part_base[KDV_MAX_BATCH];   // first workspace partial row of request b
+  int32_t v16_base[KDV_MAX_BATCH];    // first fp16 latent row of request b (TC kernel)
 };
 
 enum OutMode : int32_t { OUT_DIRECT = 0, OUT_PARTIALS = 1, OUT_WORKSPACE = 2 };
@@ -79,7 +80,14 @@ cudaError_t launch_mask_build(const int32_t* parent, const int32_t* tree_off, in
                               cudaStream_t stream);
 cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t dtype,
                                cudaStream_t stream);
-cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream);
+// v16: the fp16 latent rows written by launch_latent_f16 (request b's key j
+// at row v16_base[b] + j).
+cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const void* v16, int64_t v16_rows,
+                              cudaStream_t stream);
+// Writes the fp16 latent rows (v16, nullable) and, for a paged pool, the
+// staged bf16 rows with their offsets (staged / staged_off, nullable).
+cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v16, void* staged, int32_t* staged_off,
+                              cudaStream_t stream);
 // Work items (4-CTA clusters) of the TC kernel that fit on the device at
 // once, i.e. one wave; 0 when the query fails (no device).
 int tc2_max_active_clusters();

@@ -1,0 +1,123 @@
+// latent_f16.cu -- the fp16 copy of the latent rows that the tensor-core
+// kernel's P.V reads.
+//
+// The tensor-core verify kernel rounds the softmax numerators P to fp16 before
+// P.V (in bf16 their rounding alone would cost ~1e-3 of the output's RMS), and
+// a kind::f16 MMA needs V in the same type. Converting V inside the kernel is
+// not an option on this part: while the tensor core streams shared memory,
+// the load/store unit gets only ~5-10 B/clk of it, so a 16 KB stage read back
+// through registers takes over a microsecond. This kernel therefore writes,
+// before the verify launch, the c_kv part of every key the call will read --
+// request b's logical keys 0 .. L_b+T_b-1, through the page table when there
+// is one -- as fp16 rows [512] in logical order into the workspace, where the
+// verify kernel's P.V side reads them with tiled TMA boxes. bf16 -> fp16 is
+// exact for 2^-14 <= |x| < 65536; smaller values round to fp16 subnormals;
+// |x| >= 65536 (or inf / NaN) is reported as KDV_DERR_RANGE.
+//
+// A paged pool can also be staged in the same pass: with `staged` given, the
+// whole bf16 row (c_kv || k_rope, 1152 bytes) is copied to staged row
+// v16_base[b] + j as well, and staged_off[b] = v16_base[b], so the verify
+// kernel reads the request's keys with tiled TMA boxes instead of gathers.
+//
+// HBM-bound: 1 KB read and 1 KB written per key (+1152 B written when
+// staging). One warp per key row, lane l owning dims [16 l, 16 l + 16) (and,
+// for lanes 0-7, k_rope bytes [16 l, 16 l + 16)); each warp keeps four rows'
+// loads in flight.
+#include <cuda_fp16.h>
+
+#include "kdv_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace kdv {
+namespace {
+
+constexpr int LF_THREADS = 256;
+constexpr int LF_ROWS = 4;           // rows in flight per warp
+
+__global__ void __launch_bounds__(LF_THREADS)
+latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v16, uint8_t* __restrict__ staged,
+                  int32_t* __restrict__ staged_off) {
+  const int b = blockIdx.y;
+  if (staged_off != nullptr && blockIdx.x == 0 && b == 0)
+    for (int i = threadIdx.x; i <= p.B; i += LF_THREADS)
+      staged_off[i] = i < p.B ? p.v16_base[i] : p.v16_base[p.B - 1] + p.L[p.B - 1] + p.T[p.B - 1];
+  const int n = p.L[b] + p.T[b];
+  const int64_t kv_base = a.kv_off[b];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wstride = gridDim.x * (LF_THREADS / 32);
+  const char* kv = static_cast<const char*>(a.kv);
+  uint32_t range = 0;
+  bool bad_row = false;
+  for (int j0 = (blockIdx.x * (LF_THREADS / 32) + warp) * LF_ROWS; j0 < n; j0 += wstride * LF_ROWS) {
+    uint4 x[LF_ROWS][2], xr[LF_ROWS];
+#pragma unroll
+    for (int r = 0; r < LF_ROWS; ++r) {
+      x[r][0] = x[r][1] = xr[r] = make_uint4(0u, 0u, 0u, 0u);
+      const int j = j0 + r;
+      if (j < n) {
+        int64_t row = a.page_table != nullptr ? (int64_t)a.page_table[kv_base + j] : kv_base + j;
+        if (row < 0 || row >= a.num_slots) {
+          bad_row = true;
+          continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(kv + row * (int64_t)((a.D_c + a.D_r) * 2) + lane * 32);
+        x[r][0] = ptx::ldg_nc_v4(src);
+        x[r][1] = ptx::ldg_nc_v4(src + 1);
+        if (staged != nullptr && lane < 8)
+          xr[r] = ptx::ldg_nc_v4(reinterpret_cast<const uint4*>(kv + row * (int64_t)((a.D_c + a.D_r) * 2) + 1024 +
+                                                                   lane * 16));
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < LF_ROWS; ++r) {
+      const int j = j0 + r;
+      if (j < n) {
+        uint4 y[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 w = x[r][h];
+          range |= ptx::bf16x2_beyond_f16(w.x) | ptx::bf16x2_beyond_f16(w.y) | ptx::bf16x2_beyond_f16(w.z) |
+                   ptx::bf16x2_beyond_f16(w.w);
+          y[h] = make_uint4(ptx::bf16x2_to_f16x2(w.x), ptx::bf16x2_to_f16x2(w.y), ptx::bf16x2_to_f16x2(w.z),
+                            ptx::bf16x2_to_f16x2(w.w));
+        }
+        const int64_t out_row = (int64_t)p.v16_base[b] + j;
+        if (v16 != nullptr) {
+          uint4* dst = reinterpret_cast<uint4*>(v16 + out_row * 512 + lane * 16);
+          dst[0] = y[0];
+          dst[1] = y[1];
+        }
+        if (staged != nullptr) {
+          uint4* srow = reinterpret_cast<uint4*>(staged + out_row * (int64_t)((a.D_c + a.D_r) * 2));
+          srow[2 * lane] = x[r][0];
+          srow[2 * lane + 1] = x[r][1];
+          if (lane < 8) srow[64 + lane] = xr[r];
+        }
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, range != 0) && lane == 0) record_error(a.d_err, KDV_DERR_RANGE);
+  if (__any_sync(0xffffffffu, bad_row) && lane == 0)
+    record_error(a.d_err, a.page_table != nullptr ? KDV_DERR_BAD_SLOT : KDV_DERR_BAD_LENGTH);
+}
+
+}  // namespace
+
+cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v16, void* staged, int32_t* staged_off,
+                              cudaStream_t stream) {
+  if (a.D_c != 512 || (staged != nullptr && a.D_r != 64)) return cudaErrorInvalidValue;
+  int max_n = 0;
+  for (int b = 0; b < p.B; ++b) max_n = max_n > p.L[b] + p.T[b] ? max_n : p.L[b] + p.T[b];
+  if (max_n == 0) return cudaSuccess;
+  const int rows_per_cta = (LF_THREADS / 32) * LF_ROWS;
+  // enough CTAs in flight to keep HBM busy, fewer for a short request
+  int gx = (max_n + rows_per_cta - 1) / rows_per_cta;
+  const int cap = (8 * 148 + p.B - 1) / p.B;
+  if (gx > cap) gx = cap < 1 ? 1 : cap;
+  const dim3 grid((unsigned)gx, (unsigned)p.B);
+  latent_f16_kernel<<<grid, LF_THREADS, 0, stream>>>(a, p, static_cast<__half*>(v16), static_cast<uint8_t*>(staged),
+                                                      staged_off);
+  return cudaGetLastError();
+}
+
+}  // namespace kdv

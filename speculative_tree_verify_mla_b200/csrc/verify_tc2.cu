@@ -29,23 +29,21 @@
 //   CTA 2 + CTA 3 ("O pair"): O += P V with M=256, N=256 (two MMAs per 16
 //     keys), K=16, per 128-key P tile. O (128 rows x 512 fp32) fills each
 //     CTA's TMEM; each CTA stages 256 of the 512 V dims (the half of each
-//     N=256 column range the MMA expects from it) through a 16 KB x 6 ring.
-//     Each CTA's producer warp brings its V blocks in with TMA (tiled boxes,
-//     or four-row gathers through a page table), and four converter warps
-//     then re-encode each landed stage in place from bf16 to fp16 (see
-//     below), writing zeros for keys past the split's end so that nothing
-//     of the rows beyond it reaches P.V. CTA 2 issues the MMAs.
+//     N=256 column range the MMA expects from it) through a 16 KB x 6 ring,
+//     with TMA boxes from the call's fp16 copy of the latent rows (below).
+//     CTA 2 issues the MMAs.
 //
 // Precision of P.V. The softmax numerators P are rounded to a 16-bit type
 // before the P.V MMA, and that rounding is the kernel's dominant error. In
 // bf16 (8 significant bits) it leaves a normalised mean error near 1e-3 of
 // the output's RMS; in fp16 (11 bits) about 1.3e-4. A kind::f16 MMA takes A
-// and B of one type, so V is staged as fp16 too: bf16 -> fp16 is exact for
-// every latent value with 2^-14 <= |x| < 65536 (both types keep the 8
-// significant bits), rounds smaller values to fp16 subnormals (an absolute
-// error below 2^-25), and cannot represent |x| >= 65536, which the
-// converters report as KDV_DERR_RANGE. P is at most 2^TAU = 256 by the lazy
-// rescale rule, well inside fp16's range.
+// and B of one type, so V is read as fp16 too, from rows that
+// latent_f16.cu writes before this kernel runs (bf16 -> fp16 is exact for
+// every latent value with 2^-14 <= |x| < 65536). V cannot be converted here:
+// while the tensor core streams shared memory the load/store unit gets only
+// ~5-10 B/clk of it (measured), so reading a 16 KB stage back through
+// registers would take over a microsecond. P is at most 2^TAU = 256 by the
+// lazy rescale rule, well inside fp16's range.
 //
 // Every MMA is N=256: with the TMA stream running beside it, N=128 MMAs on
 // this part leave ~35 cycles per instruction unhidden, N=256 ones do not
@@ -107,15 +105,13 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + QK_BLOCKS * QBLOCK_BYTES;
 constexpr int OFF_XCHG = OFF_KV + KV_STAGES * KBLOCK_BYTES;   // float [2][2][128] + [128] (S side)
 constexpr int XCHG_BYTES = 5 * ROWS * 4;
-constexpr int OFF_KSLOT = OFF_XCHG + XCHG_BYTES;             // int32 [128] (S side, paged KV)
 constexpr int OFF_VRING = 0;
 constexpr int OFF_P = OFF_VRING + V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
-constexpr int OFF_VSLOT = OFF_STATS + STATS_BYTES;            // int32 [256] (O side, paged KV)
 constexpr int EPI_STAGE_BYTES = 16384;                         // per epilogue warp, over V ring + P slots
 static_assert(OFF_VRING + 8 * EPI_STAGE_BYTES <= OFF_STATS, "epilogue staging overlaps the row statistics");
-constexpr int OFF_MISC = OFF_KSLOT + HKEYS * 4;
-static_assert(OFF_VSLOT + STILE * 4 <= OFF_MISC, "O-side buffers overlap misc");
+constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
+static_assert(OFF_STATS + STATS_BYTES <= OFF_MISC, "O-side buffers overlap misc");
 constexpr int OFF_BAR = OFF_MISC;
 constexpr int NUM_BARS = 56;
 constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
@@ -134,12 +130,11 @@ static_assert(SMEM_BYTES <= 232448, "exceeds 227 KB of shared memory");
 constexpr int B_KV_FULL = 0, B_KV_EMPTY = B_KV_FULL + KV_STAGES, B_S_FULL = B_KV_EMPTY + KV_STAGES,
               B_S_EMPTY = B_S_FULL + 2, B_P_EMPTY = B_S_EMPTY + 2, B_Q_FULL = B_P_EMPTY + NP,
               B_S_DRAIN = B_Q_FULL + QK_BLOCKS;
-// O pair. V_FULL, READY and O_DRAIN in CTA 2 only; V_LANDED (a stage's TMA
-// bytes are in this CTA) and V_EMPTY in both.
+// O pair. V_FULL, READY and O_DRAIN in CTA 2 only.
 constexpr int B_V_FULL = B_S_DRAIN + 1, B_V_EMPTY = B_V_FULL + V_STAGES, B_P_FULL = B_V_EMPTY + V_STAGES,
               B_READY = B_P_FULL + NP, B_PV_DONE = B_READY + NP, B_STATS = B_PV_DONE + NP,
-              B_O_DRAIN = B_STATS + 1, B_V_LANDED = B_O_DRAIN + 1;
-static_assert(B_V_LANDED + V_STAGES <= NUM_BARS, "barrier slots");
+              B_O_DRAIN = B_STATS + 1;
+static_assert(B_O_DRAIN < NUM_BARS, "barrier slots");
 
 constexpr uint16_t S_PAIR = 0x3, O_PAIR = 0xC;     // cluster CTA masks
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(256, 256, false, false);
@@ -147,8 +142,7 @@ constexpr uint32_t IDESC_PV = idesc_f16_f32(256, 256, false, true);   // fp16 P 
 
 constexpr int THREADS = 384;
 constexpr int WG_FIRST_WARP = 4;      // warps 4-7: softmax keys 0-127 / O-side rescale + epilogue
-constexpr int WG2_FIRST_WARP = 8;     // warps 8-11: softmax keys 128-255 (S side) / V converters (O side)
-constexpr int CONVERTERS = 4;         // O-side converter warps per CTA
+constexpr int WG2_FIRST_WARP = 8;     // warps 8-11: softmax keys 128-255 (S side)
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -279,9 +273,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
     reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR)[0] = 0;
     if (s_side) {
       for (int i = 0; i < KV_STAGES; ++i) {
-        // TMA: the leader's expect_tx arrival (bytes of both CTAs counted);
-        // paged cp.async: one arrival from each CTA's producer
-        mbar_init(c.bar(B_KV_FULL + i), PAGED ? 2 : 1);
+        mbar_init(c.bar(B_KV_FULL + i), 1);              // the leader's expect_tx (both CTAs' bytes)
         mbar_init(c.bar(B_KV_EMPTY + i), 1);
       }
       for (int i = 0; i < 2; ++i) {
@@ -295,9 +287,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       tma_prefetch_desc(&tmap_q);
     } else {
       for (int i = 0; i < V_STAGES; ++i) {
-        mbar_init(c.bar(B_V_FULL + i), 2 * CONVERTERS);   // the converter warps of both O CTAs
+        mbar_init(c.bar(B_V_FULL + i), 1);               // the leader's expect_tx (both CTAs' bytes)
         mbar_init(c.bar(B_V_EMPTY + i), 1);
-        mbar_init(c.bar(B_V_LANDED + i), PAGED ? 32 : 1);   // TMA bytes, or each producer lane's copies
       }
       for (int i = 0; i < NP; ++i) {
         mbar_init(c.bar(B_P_FULL + i), 1);
@@ -335,25 +326,16 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // (nine K-blocks, kept for the whole item) and its 128 of every 256 KV
       // rows, one K-block per ring stage; everything counts on the leader's
       // barriers. Contiguous KV: TMA boxes, and the next tile's rows are
-      // prefetched into L2 while this tile streams. Paged KV: the whole warp
-      // copies each stage with 16-byte cp.async (eight lanes per pool row,
-      // four rows per instruction) into the same swizzled layout, retires it
-      // three stages later (cp.async.wait_group), orders it for the tensor
-      // core's async-proxy reads and tells the leader with one arrival.
+      // prefetched into L2 while this tile streams. Paged KV: TMA four-row
+      // gathers through the page table, lane l taking keys 4l..4l+3 of the
+      // CTA's 128 (plain loads or cp.async would go through the load/store
+      // unit, which the streaming tensor core leaves only a few B/clk of
+      // shared-memory bandwidth).
       const int n_stg = n_stiles * QK_BLOCKS;
       int issued = 0;
       // paged KV: lane l looks up keys 4l..4l+3 of this CTA's 128 one tile
-      // ahead (so the page-table latency stays off the path) and publishes
-      // them in a shared table when the tile starts
-      int32_t nslot[4] = {0, 0, 0, 0};
-      int32_t* kslot = reinterpret_cast<int32_t*>(smem + OFF_KSLOT);
-      const char* kv_bytes = static_cast<const char*>(a.kv);
-      // paged KV: stage g's copies are retired and announced to the leader
-      auto announce = [&](int g) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) arrive_on(c.bar(B_KV_FULL + g % KV_STAGES), lead_rank, rank);
-      };
+      // ahead, so the page-table latency stays off the path
+      int32_t slot[4] = {0, 0, 0, 0}, nslot[4] = {0, 0, 0, 0};
       if (PAGED && n_stiles > 0) {
         const int j0 = stile_key(0) + (int)half * HKEYS + 4 * lane;
 #pragma unroll
@@ -379,32 +361,20 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           break;
         const int tile = g / QK_BLOCKS, blk = g % QK_BLOCKS;
         const uint32_t dst = base + OFF_KV + st * KBLOCK_BYTES;
+        if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
+        const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
         if (PAGED) {
           if (blk == 0) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) kslot[4 * lane + q] = nslot[q];
-            __syncwarp();
+            for (int q = 0; q < 4; ++q) slot[q] = nslot[q];
             if (tile + 1 < n_stiles) {
               const int j0 = stile_key(tile + 1) + (int)half * HKEYS + 4 * lane;
 #pragma unroll
               for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
             }
           }
-          const int ch = lane & 7;
-#pragma unroll 4
-          for (int i = 0; i < HKEYS / 4; ++i) {
-            const int r = 4 * i + (lane >> 3);
-            cp_async16(dst + r * 128 + ((ch ^ (r & 7)) << 4),
-                       kv_bytes + (int64_t)kslot[r] * (DQ * 2) + blk * 128 + ch * 16);
-          }
-          cp_async_commit();
-          if (g >= KV_STAGES - 1) {
-            cp_async_wait<KV_STAGES - 1>();
-            announce(g - (KV_STAGES - 1));
-          }
+          tma_gather4_pair(dst + lane * 512, &tmap_kv, fb, blk * 64, slot[0], slot[1], slot[2], slot[3]);
         } else {
-          if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
-          const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
           const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
           if (blk == 0 && tile + 1 < n_stiles)
             for (int e = 0; e < QK_BLOCKS; ++e) tma_prefetch_l2(&tmap_kv, e * 64, y + STILE);
@@ -412,18 +382,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         }
         issued = g + 1;
       }
-      if (PAGED) {
-        // retire this CTA's own copies; announce the stages not yet announced
-        cp_async_wait<0>();
-        for (int g = max(0, issued - (KV_STAGES - 1)); g < issued; ++g) announce(g);
-      }
       if (leader && lane == 0) {
-        // retire copies in flight (TMA: both halves count on the leader's barriers)
+        // retire copies in flight (both halves count on the leader's barriers)
         if (n_stiles > 0)
           for (int blk = 0; blk < QK_BLOCKS; ++blk) wait_bar(c, c.bar(B_Q_FULL + blk), 0, true);
-        if (!PAGED)
-          for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
-            wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
+        for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
+          wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
       }
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T,
@@ -589,65 +553,33 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
     }
   } else {
     // ======================================================= O pair
-    if (warp == 0 && (PAGED || lane == 0)) {
-      // ---------------- V producer (both O CTAs): this CTA's 256 dims of
-      // every 32 keys, landing on this CTA's own V_LANDED barrier; local
-      // block lb holds dims 64*((lb/2)*4 + half*2 + lb%2), bf16, 128B-swizzled.
-      // Paged KV: the whole warp copies with 16-byte cp.async, one key's four
-      // 128-byte blocks per instruction, and each lane's copies arrive on
-      // V_LANDED when they complete.
+    if (warp == 0 && lane == 0) {
+      // ---------------- V producer (both O CTAs): this CTA's 256 of the 512
+      // fp16 dims of every 32 keys, read from the call's fp16 latent rows
+      // (contiguous per request, whatever the pool's layout) and counted on
+      // the leader's V_FULL; local block lb holds dims
+      // 64*((lb/2)*4 + half*2 + lb%2), 128B-swizzled. Rows past the request's
+      // keys are other requests' rows or past the end (read as zeros): finite
+      // either way, and masked out by P = 0.
       int issued = 0;
       const int n_sub = (STILE / VKEYS) * n_stiles;
-      // paged KV: the 256 slots of an S tile sit in a shared table (lane l
-      // reads keys 8l..8l+7 of the next tile one tile ahead, in registers)
-      int32_t* vslot = reinterpret_cast<int32_t*>(smem + OFF_VSLOT);
-      int32_t nv[8];
-      if (PAGED && n_stiles > 0) {
-#pragma unroll
-        for (int m = 0; m < 8; ++m) nv[m] = paged_slot(a, kv_base, stile_key(0) + 8 * lane + m, k_hi);
-      }
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
-        const uint32_t eparity = ((u / V_STAGES) & 1) ^ 1;
-        if (!(PAGED ? wait_warp(c, c.bar(B_V_EMPTY + st), eparity, true)
-                    : wait_bar(c, c.bar(B_V_EMPTY + st), eparity, true)))
-          break;
-        const uint32_t lb_bar = c.bar(B_V_LANDED + st);
-        if (!PAGED && lane == 0) mbar_arrive_expect_tx(lb_bar, V_STAGE_BYTES);
+        if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1, true)) break;
+        if (leader) mbar_arrive_expect_tx(c.bar(B_V_FULL + st), 2 * V_STAGE_BYTES);
         const int key0 = stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS;
         const uint32_t dst = base + OFF_VRING + st * V_STAGE_BYTES;
-        if (PAGED) {
-          const int vt = u / (STILE / VKEYS);
-          if (u % (STILE / VKEYS) == 0) {          // entering S tile vt: publish its slots
-#pragma unroll
-            for (int m = 0; m < 8; ++m) vslot[8 * lane + m] = nv[m];
-            if (vt + 1 < n_stiles) {
-#pragma unroll
-              for (int m = 0; m < 8; ++m) nv[m] = paged_slot(a, kv_base, stile_key(vt + 1) + 8 * lane + m, k_hi);
-            }
-            __syncwarp();
-          }
-          const int lb = lane >> 3, ch = lane & 7;
+        const uint32_t fb = mapa(c.bar(B_V_FULL + st), lead_rank);
+        const int32_t y = p.v16_base[b] + key0;
+        for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
           const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-          const char* src0 = static_cast<const char*>(a.kv) + gb * 128 + ch * 16;
-          const int k0 = key0 - stile_key(vt);
-#pragma unroll 4
-          for (int k = 0; k < VKEYS; ++k)
-            cp_async16(dst + lb * VBLOCK_BYTES + k * 128 + ((ch ^ (k & 7)) << 4),
-                       src0 + (int64_t)vslot[k0 + k] * (DQ * 2));
-          cp_async_arrive_noinc(lb_bar);
-        } else {
-          const int32_t y = (int32_t)(kv_base + key0);
-          for (int lb = 0; lb < V_LOCAL_BLOCKS; ++lb) {
-            const int gb = (lb >> 1) * 4 + (int)half * 2 + (lb & 1);
-            tma_load_2d(dst + lb * VBLOCK_BYTES, &tmap_v, lb_bar, gb * 64, y);
-          }
+          tma_load_2d_pair(dst + lb * VBLOCK_BYTES, &tmap_v, fb, gb * 64, y);
         }
         issued = u + 1;
       }
-      if (lane == 0)
+      if (leader)
         for (int u = max(0, issued - V_STAGES); u < issued; ++u)
-          wait_bar(c, c.bar(B_V_LANDED + u % V_STAGES), (u / V_STAGES) & 1, true);
+          wait_bar(c, c.bar(B_V_FULL + u % V_STAGES), (u / V_STAGES) & 1, true);
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------- pair MMA issuer: O[256 x 512] += P[256 x 128] . V[128 x 512]
       for (int i = 0; i < n_ptiles; ++i) {
@@ -750,52 +682,6 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           tear[1 + sp] = (uint32_t)first_miss;
           tear[5 + sp] = got_stats ? 1u : 0u;
         }
-      } else {
-        // ---------------- V converters (warps 8-11, both O CTAs): once stage
-        // u's TMA bytes have landed in this CTA, re-encode its 16 KB in place
-        // from bf16 to fp16 (every 16-byte chunk keeps its place; the chunk at
-        // byte b holds 8 dims of key b % 4096 / 128 of the stage), write
-        // zeros for keys at or past the split's end, and tell the MMA issuer.
-        // Thread t takes chunks t, t + 128, ...: a warp covers 512 contiguous
-        // bytes per access.
-        const int tid = (warp - WG2_FIRST_WARP) * 32 + lane;
-        const int n_sub = (STILE / VKEYS) * n_stiles;
-        const uint32_t vfull_lead = mapa(c.bar(B_V_FULL), lead_rank);
-        uint32_t range = 0;
-        bool ok = true;
-        for (int u = 0; ok && u < n_sub; ++u) {
-          const int st = u % V_STAGES;
-          ok = wait_warp(c, c.bar(B_V_LANDED + st), (u / V_STAGES) & 1);
-          if (!ok) break;
-          const int live = k_hi - (stile_key(u / (STILE / VKEYS)) + (u % (STILE / VKEYS)) * VKEYS);
-          const uint32_t sb = base + OFF_VRING + st * V_STAGE_BYTES;
-#pragma unroll
-          for (int i = 0; i < V_STAGE_BYTES / 16 / (32 * CONVERTERS); ++i) {
-            const uint32_t off = (uint32_t)(tid + 32 * CONVERTERS * i) * 16u;
-            const uint32_t addr = sb + off;
-            uint4 v;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-            if ((int)((off & (VBLOCK_BYTES - 1)) >> 7) < live) {
-              range |= bf16x2_beyond_f16(v.x) | bf16x2_beyond_f16(v.y) | bf16x2_beyond_f16(v.z) |
-                       bf16x2_beyond_f16(v.w);
-              v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
-            } else {
-              v = make_uint4(0u, 0u, 0u, 0u);
-            }
-            st_shared_v4(addr, v.x, v.y, v.z, v.w);
-          }
-          // the pair's MMA reads these bytes through the async proxy: every
-          // thread orders its stores before async-proxy reads, then one
-          // relaxed arrive per warp (as for the P tiles; a release-ordered
-          // remote arrive would stall the warp ~1800 cycles per stage)
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (leader) mbar_arrive(c.bar(B_V_FULL + st));
-            else mbar_arrive_remote_relaxed(vfull_lead + st * 8);
-          }
-        }
-        if (__any_sync(0xffffffffu, range != 0) && lane == 0) record_error(a.d_err, KDV_DERR_RANGE);
       }
       // warps 8-11 learn of the final MMA and the statistics through this barrier
       bad = named_bar_or(1, 2 * 128, bad);
@@ -935,7 +821,8 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStream_t stream) {
+cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const void* v16, int64_t v16_rows,
+                              cudaStream_t stream) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   if (a.num_slots < 1 || a.num_slots > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
@@ -951,9 +838,19 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, cudaStre
   };
   CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o;
   const bool paged = a.page_table != nullptr;
-  // paged KV: one-row boxes for the K and V gathers
+  if (v16 == nullptr || v16_rows < 1 || v16_rows > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
+  // V: the fp16 latent rows [v16_rows][512] in 32-row boxes
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)DC, (cuuint64_t)v16_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)DC * 2};
+    const cuuint32_t box[2] = {64, VKEYS};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmap_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(v16), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : HKEYS) != CUDA_SUCCESS ||
-      make(&tmap_v, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : VKEYS) != CUDA_SUCCESS ||
       make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   // output rows for the epilogue's TMA stores

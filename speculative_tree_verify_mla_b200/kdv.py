@@ -45,7 +45,7 @@ KDV_MAX_BATCH = 128
 # Every entry point include/kdv.h declares (checked by the CPU tests).
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
-            "kdv_verify_attn_noalloc", "kdv_combine", "kdv_tree_accept_workspace",
+            "kdv_verify_attn_noalloc", "kdv_latent_f16", "kdv_combine", "kdv_tree_accept_workspace",
             "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o", "kdv_tree_build")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -73,7 +73,7 @@ class VerifyParams(ctypes.Structure):
         ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
         ("o_part", ctypes.c_void_p), ("lse_part", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-        ("d_err", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64),
+        ("d_err", ctypes.c_void_p), ("wait_limit_ns", ctypes.c_uint64), ("v16", ctypes.c_void_p),
     ]
 
 
@@ -132,6 +132,8 @@ def load() -> ctypes.CDLL:
         lib.kdv_verify_attn.restype = c.c_int
         lib.kdv_verify_attn_noalloc.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
         lib.kdv_verify_attn_noalloc.restype = c.c_int
+        lib.kdv_latent_f16.argtypes = [c.POINTER(VerifyParams), c.c_void_p, c.c_void_p]
+        lib.kdv_latent_f16.restype = c.c_int
         lib.kdv_combine.argtypes = [c.c_void_p, c.c_void_p, c.c_int32, c.c_int64, c.c_int32,
                                     c.c_void_p, c.c_void_p, c.c_void_p]
         lib.kdv_combine.restype = c.c_int
@@ -233,6 +235,11 @@ def kdv_verify_attn_noalloc(params: VerifyParams, stream=None) -> None:
     """kdv_verify_attn with the library's built-in scratch instead of params.workspace."""
     _check(load().kdv_verify_attn_noalloc(ctypes.byref(params), _stream(stream)),
            "kdv_verify_attn_noalloc")
+
+
+def kdv_latent_f16(params: VerifyParams, v16: torch.Tensor, stream=None) -> None:
+    """The fp16 latent rows [sum(L+T)][512] of a call (see kdv.h)."""
+    _check(load().kdv_latent_f16(ctypes.byref(params), _ptr(v16), _stream(stream)), "kdv_latent_f16")
 
 
 def _dt(t: torch.Tensor) -> int:

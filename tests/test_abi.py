@@ -38,7 +38,7 @@ def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4):
         assert kdv.status_string(s).startswith("KDV_")
     assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
-    assert kdv.kdv_version() == 110
+    assert kdv.kdv_version() == 120
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
@@ -65,7 +65,7 @@ def _params(**over):
                 page_table=None, kv_off=None, tree_off=None, prefix_len=None,
                 h_prefix_len=[5], h_tree_T=[3], mask=None, num_splits=0, return_partials=0,
                 o=None, lse=None, o_part=None, lse_part=None, workspace=None,
-                workspace_bytes=0, d_err=None)
+                workspace_bytes=0, d_err=None, v16=None)
     base.update(over)
     return kdv.make_params(**base)
 
@@ -119,10 +119,18 @@ def test_workspace_sizes(lib):
     n = kdv.kdv_verify_attn_workspace(_params(num_splits=3))
     parts = 3 * 3 * 4
     assert n == ((parts * 64 * 4 + 255) // 256) * 256 + parts * 4
-    # the tensor-core kernel keeps its merge partials o_k in fp16
+    # the tensor-core kernel keeps its merge partials o_k in fp16, then the
+    # fp16 latent rows of every key the call reads (L + T = 8 here, 1 KB each)
+    al = lambda x: ((x + 255) // 256) * 256
     p = _params(num_splits=3, dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC)
     n = kdv.kdv_verify_attn_workspace(p)
-    assert n == ((parts * 512 * 2 + 255) // 256) * 256 + parts * 4
+    assert n == al(al(parts * 512 * 2) + parts * 4) + al(8 * 1024)
+    # ... unless the caller passes those rows
+    p = _params(num_splits=3, dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC, v16=0x10000)
+    assert kdv.kdv_verify_attn_workspace(p) == al(parts * 512 * 2) + parts * 4
+    # a single split: only the fp16 rows
+    p = _params(num_splits=1, dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC)
+    assert kdv.kdv_verify_attn_workspace(p) == al(8 * 1024)
     # partials returned to the caller: no workspace
     assert kdv.kdv_verify_attn_workspace(_params(num_splits=3, return_partials=1)) == 0
 
@@ -240,14 +248,16 @@ def test_tree_build_validation(lib):
 
 
 def test_staged_workspace_size(lib):
-    # forced single split (no merge region): staged offsets [B+1] then the rows
+    al = lambda x: ((x + 255) // 256) * 256
+    # forced single split (no merge region): the fp16 latent rows, then the
+    # staged offsets [B+1], then the staged rows
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC_STAGED,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
-    assert kdv.kdv_verify_attn_workspace(p) == 256 + 103 * 576 * 2
-    # the gather path needs none
+    assert kdv.kdv_verify_attn_workspace(p) == al(103 * 1024) + 256 + 103 * 576 * 2
+    # reading the pool through the page table needs only the fp16 rows
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
-    assert kdv.kdv_verify_attn_workspace(p) == 0
+    assert kdv.kdv_verify_attn_workspace(p) == al(103 * 1024)
     # impl codes past the last one are rejected
     n = ctypes.c_size_t(0)
     assert lib.kdv_verify_attn_workspace(ctypes.byref(_params(impl=5)), ctypes.byref(n)) == \

@@ -131,16 +131,19 @@ def test_tc_paged_bad_slot_reported():
     assert dc.error_flag() == kdv.KDV_DERR_BAD_SLOT
 
 
-def test_tc_auto_picks_tc_for_paged():
-    case = datagen.make_case("ap", **datagen.KIMI, prefix_len=[100],
+def test_tc_auto_stages_a_paged_pool():
+    """AUTO reads a paged pool through the staged contiguous copy (its
+    workspace covers it), and gives the bits the in-place gathers give."""
+    case = datagen.make_case("ap", **datagen.KIMI, prefix_len=[1000],
                              parents=[datagen.chain_tree(3)], seed=2, paged=True)
     dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_AUTO, num_splits=0)
-    plan = kdv.kdv_verify_attn_plan(dc.params)
+    dc_st = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_STAGED, num_splits=0)
     dc_tc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC, num_splits=0)
-    assert plan == kdv.kdv_verify_attn_plan(dc_tc.params)
+    assert dc.ws_bytes == dc_st.ws_bytes > dc_tc.ws_bytes
     o, lse = dc.run().results()
     o2, lse2 = dc_tc.run().results()
     np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, lse2)
 
 
 
