@@ -150,34 +150,54 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" :: "r"(addr), "r"(v) : "memory");
+}
+
+// Per-CTA wait context. It must stay in registers: a copy in local memory
+// (which a reference passed to an out-of-line function forces) turns every
+// wait into a load through the load/store unit, which the streaming tensor
+// core leaves a few B/clk of the SM's shared-memory/L1 bandwidth -- enough to
+// stall the MMA issuer hundreds of cycles per ring stage.
 struct Ctx {
   uint32_t base;
-  volatile uint32_t* abort_flag;
   int32_t* d_err;
   uint64_t limit;        // ns a pipeline wait may take (drain waits always get TIMEOUT_NS)
   __device__ uint32_t bar(int i) const { return base + OFF_BAR + 8 * i; }
+  __device__ uint32_t abort_addr() const { return base + OFF_ABORT; }
 };
+
+// The part of a bounded wait that runs once the first probe failed: it takes
+// scalars only, so calling it out of line keeps nothing of the caller in memory.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, uint32_t abort_addr, int32_t* d_err,
+                                           uint64_t lim, bool drain) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (!drain && ld_shared_u32(abort_addr) != 0) return false;
+      if (globaltimer() - t0 > lim) {
+        st_shared_u32(abort_addr, 1u);
+        record_error(d_err, KDV_DERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
 
 // Bounded wait for phase `parity` of `bar`. A pipeline wait gives up after
 // c.limit ns (recording KDV_DERR_TIMEOUT and raising this CTA's abort flag)
 // or as soon as the flag is up; a drain wait -- one that retires this CTA's
 // own copies and MMAs before it exits -- ignores the flag and waits up to
 // TIMEOUT_NS.
-__device__ __noinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
+__device__ __forceinline__ bool wait_bar(const Ctx& c, uint32_t bar, uint32_t parity, bool drain = false) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  const uint64_t lim = drain ? TIMEOUT_NS : c.limit;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (!drain && *c.abort_flag) return false;
-      if (globaltimer() - t0 > lim) {
-        *c.abort_flag = 1;
-        record_error(c.d_err, KDV_DERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
+  return wait_bar_slow(bar, parity, c.abort_addr(), c.d_err, drain ? TIMEOUT_NS : c.limit, drain);
 }
 
 // Wait for phase `parity` of `bar` until the globaltimer reaches `deadline`.
@@ -246,7 +266,6 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 
   Ctx c;
   c.base = base;
-  c.abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_ABORT);
   c.d_err = a.d_err;
   c.limit = a.wait_limit_ns > 0 ? a.wait_limit_ns : TIMEOUT_NS;
 
@@ -269,7 +288,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 
   // ---- setup -------------------------------------------------------------
   if (threadIdx.x == 0) {
-    *c.abort_flag = 0;
+    st_shared_u32(c.abort_addr(), 0u);
     reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR)[0] = 0;
     if (s_side) {
       for (int i = 0; i < KV_STAGES; ++i) {
@@ -494,11 +513,21 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             m_half = fmaxf(m_half, xk);
           }
         }
-        // row max of the whole 256-key tile from both warpgroups
-        volatile float* xm = xchg + (i & 1) * 2 * ROWS;
-        xm[hw * ROWS + r] = m_half;
-        named_bar_sync(1, 2 * 128);
-        const float m_tile = fmaxf(m_half, xm[(hw ^ 1) * ROWS + r]);
+        // Row max of the whole 256-key tile from both warpgroups -- needed
+        // only if some row's reference max may move. One barrier vote
+        // decides: when no half-tile max exceeds its row's m_run + TAU (and
+        // no row sees its first finite logit), neither does the full-tile
+        // max, so the exchange through shared memory (load/store-unit work
+        // that the streaming tensor core starves) is skipped. Either way
+        // both warpgroups take the same decision as with the exchange.
+        const bool moves = m_half > m_run + TAU || (m_run == -INFINITY && m_half != -INFINITY);
+        float m_tile = m_half;
+        if (named_bar_or(1, 2 * 128, moves)) {
+          volatile float* xm = xchg + (i & 1) * 2 * ROWS;
+          xm[hw * ROWS + r] = m_half;
+          named_bar_sync(1, 2 * 128);
+          m_tile = fmaxf(m_half, xm[(hw ^ 1) * ROWS + r]);
+        }
         float alpha = 1.f;
         if (m_tile > m_run + TAU || (m_run == -INFINITY && m_tile != -INFINITY)) {
           if (m_run != -INFINITY) {
@@ -779,7 +808,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   volatile uint32_t* tear = reinterpret_cast<volatile uint32_t*>(smem + OFF_TEAR);
   __syncwarp();
   __syncthreads();
-  if (threadIdx.x < 4 && *c.abort_flag != 0) st_cluster_u32(mapa(base + OFF_TEAR, threadIdx.x), 1u);
+  if (threadIdx.x < 4 && ld_shared_u32(c.abort_addr()) != 0) st_cluster_u32(mapa(base + OFF_TEAR, threadIdx.x), 1u);
   tc_fence_before();
   cluster_sync();
   if (tear[0] != 0) {
