@@ -81,9 +81,9 @@ constexpr int QBLOCK_BYTES = ROWS * 128;            // 128 rows x 64 dims (16 KB
 constexpr int QK_BLOCKS = DQ / 64;                  // 9 (8 latent + 1 rope)
 constexpr int V_LOCAL_BLOCKS = 4;                   // V dim-blocks per O CTA per stage
 constexpr int KV_STAGES = 4;                        // KV ring: one 16 KB K-block per stage
-constexpr int V_STAGES = 6;
+constexpr int V_STAGES = 5;
 constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
-constexpr int NP = 3;                               // P slots per O CTA
+constexpr int NP = 4;                               // P slots per O CTA (slots 2j+hw: one pair per warpgroup)
 constexpr int P_BYTES = ROWS * KEYS * 2;
 constexpr int P_KCHUNK_BYTES = ROWS * 16;           // 8 keys of all 128 rows (interleaved core matrices)
 constexpr int P_MSG_BYTES = P_BYTES + ROWS * 4;
@@ -100,7 +100,7 @@ constexpr uint64_t TIMEOUT_NS = 1000000000ull;
 //           128B-swizzled K-blocks of 64 dims (the A operand of Q.K^T, read
 //           by every tile); [147456, 212992) KV ring (4 x 16 KB, one K-block
 //           of the CTA's 128 keys per stage); row-max / row-sum exchange.
-//   O CTAs: [0, 98304) V ring (6 x 16 KB); 3 P slots; final stats.
+//   O CTAs: [0, 81920) V ring (5 x 16 KB); 4 P slots; final stats.
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + QK_BLOCKS * QBLOCK_BYTES;
 constexpr int OFF_XCHG = OFF_KV + KV_STAGES * KBLOCK_BYTES;   // float [2][2][128] + [128] (S side)
@@ -110,7 +110,7 @@ constexpr int OFF_P = OFF_VRING + V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
 constexpr int EPI_STAGE_BYTES = 16384;                         // per epilogue warp, over V ring + P slots
 static_assert(OFF_VRING + 8 * EPI_STAGE_BYTES <= OFF_STATS, "epilogue staging overlaps the row statistics");
-constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES;
+constexpr int OFF_MISC = OFF_XCHG + XCHG_BYTES > OFF_STATS + STATS_BYTES ? OFF_XCHG + XCHG_BYTES : OFF_STATS + STATS_BYTES;
 static_assert(OFF_STATS + STATS_BYTES <= OFF_MISC, "O-side buffers overlap misc");
 constexpr int OFF_BAR = OFF_MISC;
 constexpr int NUM_BARS = 56;
