@@ -360,14 +360,19 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 #pragma unroll
         for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
       }
-      if (n_stiles > 0 && lane == 0) {
-        const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
-        for (int blk = 0; blk < QK_BLOCKS; ++blk) {
-          if (leader) mbar_arrive_expect_tx(c.bar(B_Q_FULL + blk), 2 * QBLOCK_BYTES);
-          tma_load_2d_pair(base + OFF_Q + blk * QBLOCK_BYTES, &tmap_q, mapa(c.bar(B_Q_FULL + blk), lead_rank),
-                           blk * 64, qy);
-        }
-      }
+      // The query K-blocks go out interleaved with the first KV stages
+      // (q0 kv0 q1 kv1 ... q3 kv3, then q4..q8), so the first tile's MMAs
+      // start once block 0 of both has landed rather than after all of q.
+      const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
+      int q_issued = 0;
+      auto issue_q = [&](int upto) {
+        if (lane == 0)
+          for (; q_issued < upto; ++q_issued) {
+            if (leader) mbar_arrive_expect_tx(c.bar(B_Q_FULL + q_issued), 2 * QBLOCK_BYTES);
+            tma_load_2d_pair(base + OFF_Q + q_issued * QBLOCK_BYTES, &tmap_q,
+                             mapa(c.bar(B_Q_FULL + q_issued), lead_rank), q_issued * 64, qy);
+          }
+      };
       // A free ring stage is waited for like a drain (no abort check, 1 s):
       // both producers of the pair watch the same multicast commits, so they
       // issue the same stages -- the leader's drain below covers the pair's
@@ -379,6 +384,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
                     : wait_bar(c, c.bar(B_KV_EMPTY + st), eparity, true)))
           break;
         const int tile = g / QK_BLOCKS, blk = g % QK_BLOCKS;
+        if (g < KV_STAGES) issue_q(g + 1);
         const uint32_t dst = base + OFF_KV + st * KBLOCK_BYTES;
         if (leader && lane == 0) mbar_arrive_expect_tx(c.bar(B_KV_FULL + st), 2 * KBLOCK_BYTES);
         const uint32_t fb = mapa(c.bar(B_KV_FULL + st), lead_rank);
@@ -400,11 +406,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           tma_load_2d_pair(dst, &tmap_kv, fb, blk * 64, y);
         }
         issued = g + 1;
+        if (g == KV_STAGES - 1) issue_q(QK_BLOCKS);
       }
       if (leader && lane == 0) {
         // retire copies in flight (both halves count on the leader's barriers)
-        if (n_stiles > 0)
-          for (int blk = 0; blk < QK_BLOCKS; ++blk) wait_bar(c, c.bar(B_Q_FULL + blk), 0, true);
+        for (int blk = 0; blk < q_issued; ++blk) wait_bar(c, c.bar(B_Q_FULL + blk), 0, true);
         for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
           wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
       }
