@@ -384,7 +384,10 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     a.page_table = nullptr;
     a.kv_off = staged_off;
   }
-  cudaError_t e = is_tc2(impl) ? launch_verify_tc2(a, plan, v16, plan_keys(plan), s)
+  // The attention kernel may start while the latent pass still runs when
+  // that pass writes only the fp16 rows (not a staged pool the S side reads).
+  cudaError_t e = is_tc2(impl) ? launch_verify_tc2(a, plan, v16, plan_keys(plan),
+                                                   own_v16 != nullptr && staged == nullptr, s)
                                : launch_verify_simt(a, plan, p->dtype, s);
   if (e != cudaSuccess) return KDV_ERR_CUDA;
   if (plan.out_mode == OUT_WORKSPACE)

@@ -81,9 +81,12 @@ cudaError_t launch_mask_build(const int32_t* parent, const int32_t* tree_off, in
 cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t dtype,
                                cudaStream_t stream);
 // v16: the fp16 latent rows written by launch_latent_f16 (request b's key j
-// at row v16_base[b] + j).
+// at row v16_base[b] + j). after_latent: the launch right before this one on
+// `stream` is the latent pass that writes v16, and it writes nothing else
+// this kernel reads; the kernel is then launched as its programmatic
+// dependent and only the V loads wait for it (griddepcontrol.wait).
 cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const void* v16, int64_t v16_rows,
-                              cudaStream_t stream);
+                              bool after_latent, cudaStream_t stream);
 // Writes the fp16 latent rows (v16, nullable) and, for a paged pool, the
 // staged bf16 rows with their offsets (staged / staged_off, nullable).
 cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v16, void* staged, int32_t* staged_off,

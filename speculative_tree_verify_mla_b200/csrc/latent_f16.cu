@@ -38,6 +38,9 @@ __global__ void __launch_bounds__(LF_THREADS)
 latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v16, uint8_t* __restrict__ staged,
                   int32_t* __restrict__ staged_off) {
   const int b = blockIdx.y;
+  // let a dependent attention grid launch now: it waits for this grid's
+  // completion before it reads the rows (griddepcontrol.wait)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (staged_off != nullptr && blockIdx.x == 0 && b == 0)
     for (int i = threadIdx.x; i <= p.B; i += LF_THREADS)
       staged_off[i] = i < p.B ? p.v16_base[i] : p.v16_base[p.B - 1] + p.L[p.B - 1] + p.T[p.B - 1];

@@ -598,6 +598,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // either way, and masked out by P = 0.
       int issued = 0;
       const int n_sub = (STILE / VKEYS) * n_stiles;
+      // The fp16 rows may still be being written by the latent pass this
+      // grid was launched to overlap (programmatic dependent launch): wait
+      // for that grid's completion before the first V load. A no-op when the
+      // grid was launched normally.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      asm volatile("fence.proxy.async.global;" ::: "memory");
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
         if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1, true)) break;
@@ -857,7 +863,7 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const void* v16, int64_t v16_rows,
-                              cudaStream_t stream) {
+                              bool after_latent, cudaStream_t stream) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   if (a.num_slots < 1 || a.num_slots > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
@@ -916,11 +922,25 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  if (paged)
+  if (paged) {
     verify_tc2_kernel<true><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
-  else
+    return cudaGetLastError();
+  }
+  if (!after_latent) {
     verify_tc2_kernel<false><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
-  return cudaGetLastError();
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4 * p.n_items);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, verify_tc2_kernel<false>, tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
 }
 
 int tc2_max_active_clusters() {
