@@ -19,7 +19,7 @@
 //     128-255 in CTA 1), N=256 keys, K=576, both operands in shared memory.
 //     Each CTA keeps its rows' q (q_lat || q_rope, 144 KB) in shared memory
 //     for the whole item and stages the KV rows of its half of the keys (128
-//     of every 256) through a 16 KB x 4 ring, one 64-dim K-block per stage;
+//     of every 256) through a 16 KB x 5 ring, one 64-dim K-block per stage;
 //     the next tile's rows are prefetched into L2 meanwhile. TMEM holds two
 //     S buffers of 256 columns, so the MMAs of tile i+1 (issued by CTA 0)
 //     run while the softmax warps drain tile i. Two softmax warpgroups per
@@ -80,7 +80,7 @@ constexpr int VBLOCK_BYTES = VKEYS * 128;           // 32 keys x 64 dims (4 KB)
 constexpr int QBLOCK_BYTES = ROWS * 128;            // 128 rows x 64 dims (16 KB)
 constexpr int QK_BLOCKS = DQ / 64;                  // 9 (8 latent + 1 rope)
 constexpr int V_LOCAL_BLOCKS = 4;                   // V dim-blocks per O CTA per stage
-constexpr int KV_STAGES = 4;                        // KV ring: one 16 KB K-block per stage
+constexpr int KV_STAGES = 5;                        // KV ring: one 16 KB K-block per stage
 constexpr int V_STAGES = 5;
 constexpr int V_STAGE_BYTES = V_LOCAL_BLOCKS * VBLOCK_BYTES;  // 16 KB
 constexpr int NP = 4;                               // P slots per O CTA (slots 2j+hw: one pair per warpgroup)
@@ -98,13 +98,13 @@ constexpr uint64_t TIMEOUT_NS = 1000000000ull;
 // Shared-memory layout (same offsets in all four CTAs; mapa() relies on it).
 //   S CTAs: [0, 147456) the CTA's 128 query rows, q_lat || q_rope, as nine
 //           128B-swizzled K-blocks of 64 dims (the A operand of Q.K^T, read
-//           by every tile); [147456, 212992) KV ring (4 x 16 KB, one K-block
+//           by every tile); [147456, 229376) KV ring (5 x 16 KB, one K-block
 //           of the CTA's 128 keys per stage); row-max / row-sum exchange.
 //   O CTAs: [0, 81920) V ring (5 x 16 KB); 4 P slots; final stats.
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + QK_BLOCKS * QBLOCK_BYTES;
 constexpr int OFF_XCHG = OFF_KV + KV_STAGES * KBLOCK_BYTES;   // float [2][2][128] + [128] (S side)
-constexpr int XCHG_BYTES = 5 * ROWS * 4;
+constexpr int XCHG_BYTES = 3 * ROWS * 4;   // [2 hw][128] row maxima + [128] row sums
 constexpr int OFF_VRING = 0;
 constexpr int OFF_P = OFF_VRING + V_STAGES * V_STAGE_BYTES;
 constexpr int OFF_STATS = OFF_P + NP * P_SLOT_BYTES;
@@ -361,7 +361,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         for (int q = 0; q < 4; ++q) nslot[q] = paged_slot(a, kv_base, j0 + q, k_hi);
       }
       // The query K-blocks go out interleaved with the first KV stages
-      // (q0 kv0 q1 kv1 ... q3 kv3, then q4..q8), so the first tile's MMAs
+      // (q_k just before KV stage k while the ring fills, then the rest), so the first tile's MMAs
       // start once block 0 of both has landed rather than after all of q.
       const int32_t qy = (int32_t)((int64_t)p.tree_base[b] * H + row0);
       int q_issued = 0;
@@ -455,7 +455,10 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const int row = row0 + r;
       const bool valid = row < rows_b;
       const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-      float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);   // [2 parity][2 hw][128] (+ final sums)
+      // [2 hw][128] row maxima (+ [128] final sums); one buffer suffices:
+      // every tile's vote is a barrier between one exchange's reads and the
+      // next exchange's writes
+      float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);
       bool ok = true;
       const uint64_t mask_t = valid ? a.mask[p.tree_base[b] + row / H] : 0ull;
       // a warp whose 32 rows all lie past the request's last row (the tail
@@ -529,7 +532,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const bool moves = m_half > m_run + TAU || (m_run == -INFINITY && m_half != -INFINITY);
         float m_tile = m_half;
         if (named_bar_or(1, 2 * 128, moves)) {
-          volatile float* xm = xchg + (i & 1) * 2 * ROWS;
+          volatile float* xm = xchg;
           xm[hw * ROWS + r] = m_half;
           named_bar_sync(1, 2 * 128);
           m_tile = fmaxf(m_half, xm[(hw ^ 1) * ROWS + r]);
@@ -574,7 +577,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         if (ok) st_async_f32(pslot + P_BYTES + r * 4, hw == 0 ? alpha : 1.f, pbar);
       }
       // final row statistics (sum of both halves) for the O side's epilogue
-      volatile float* xs = xchg + 4 * ROWS;
+      volatile float* xs = xchg + 2 * ROWS;
       named_bar_sync(1, 2 * 128);
       if (hw == 1) xs[r] = l_part;
       named_bar_sync(1, 2 * 128);
