@@ -330,6 +330,10 @@ template <uint32_t N> __device__ __forceinline__ void regs_inc() {
 
 // Named barrier over `count` threads (count a multiple of 32). The
 // non-.aligned form: lanes of a warp may arrive at different times.
+// Arrive on named barrier `id` without waiting (the other participants sync on it).
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" :: "r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("barrier.sync %0, %1;" :: "r"(id), "r"(count) : "memory");
 }

@@ -552,7 +552,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         const uint32_t pslot = pslot0 + pslot_i * P_SLOT_BYTES;
         const uint32_t pbar = pbar0 + pslot_i * 8;
         ok = wait_warp(c, c.bar(B_P_EMPTY + pslot_i), ((pt / NP) & 1) ^ 1) && ok;
+        // The two warpgroups are staggered by half a P tile: warpgroup 1
+        // starts once warpgroup 0 has pushed its first 64 keys, so one
+        // warpgroup's exp2 work overlaps the other's DSMEM pushes instead of
+        // both computing, then both pushing.
         float lsum = 0.f;
+        if (hw == 1) named_bar_sync(2, 2 * 128);
         if (warp_rows) {
 #pragma unroll
           for (int ch = 0; ch < KEYS / 8; ++ch) {
@@ -567,10 +572,14 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
             // so a warp's 32 rows fill 512 contiguous bytes per store
             if (ok) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, w[0], w[1], w[2], w[3], pbar);
+            if (hw == 0 && ch == KEYS / 16 - 1) named_bar_arrive(2, 2 * 128);
           }
-        } else if (ok) {
+        } else {
+          if (hw == 0) named_bar_arrive(2, 2 * 128);
+          if (ok) {
 #pragma unroll 1
-          for (int ch = 0; ch < KEYS / 8; ++ch) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, 0u, 0u, 0u, 0u, pbar);
+            for (int ch = 0; ch < KEYS / 8; ++ch) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, 0u, 0u, 0u, 0u, pbar);
+          }
         }
         l_part += lsum;
         // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
