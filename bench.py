@@ -746,10 +746,11 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT)
     ap.add_argument("--impl", choices=["kdv", "reference"], default="kdv")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["auto", "tc2", "tc2s"], default="auto",
+    ap.add_argument("--kernel", choices=["auto", "tc2", "tc2s", "simt"], default="auto",
                     help="auto (default: what KDV_IMPL_AUTO picks -- the tensor-core kernel, over a "
                          "staged contiguous copy when the pool is paged), tc2 (the tensor-core "
-                         "kernel, gathering a paged pool through its page table), tc2s (staged)")
+                         "kernel, gathering a paged pool through its page table), tc2s (staged), "
+                         "simt (the CUDA-core kernel)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kimi",
                     help="kimi (default, the headline): " + WORKLOADS["kimi"] + "; sweep: "
                          + WORKLOADS["sweep"] + " (--sweep-L picks L); long: " + WORKLOADS["long"]
@@ -758,7 +759,7 @@ def parse_args(argv=None):
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the sub-records (other configurations, acceptance, projections, builder)")
     args = ap.parse_args(argv)
-    args.impl_code = {"auto": 0, "tc2": 2, "tc2s": 4}[args.kernel]
+    args.impl_code = {"auto": 0, "tc2": 2, "tc2s": 4, "simt": 1}[args.kernel]
     args.warmup = max(3, args.warmup)
     return args
 

@@ -756,38 +756,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const bool warp_full = o_tma != 0 && !bad && wrow0 + 32 <= rows_b;
       const int64_t wy = out_row_index(p, b, split, wrow0);
       const uint32_t stage = base + OFF_VRING + ew * EPI_STAGE_BYTES;
-      const int cols_per_box = p.part_f16 ? 64 : 32;
-#pragma unroll 1
-      for (int cb = 0; cb < 256 / cols_per_box; ++cb) {
-        const int col = eh * 256 + cb * cols_per_box;
-        uint32_t v[32];
-        if (p.part_f16) {
-          // two 32-column TMEM loads packed into 32 words of fp16 pairs
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t t[32];
-            if (have_o) {
-              tmem_ld32(tmem + lane_base + col + 32 * hf, t);
-              tmem_wait_ld();
-            } else {
-#pragma unroll
-              for (int k = 0; k < 32; ++k) t[k] = 0u;
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              v[16 * hf + k] = pack_f16x2(__uint_as_float(t[2 * k]) * inv, __uint_as_float(t[2 * k + 1]) * inv);
-          }
-        } else {
-          if (have_o) {
-            tmem_ld32(tmem + lane_base + col, v);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = 0u;
-          }
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * inv);
-        }
+      // 64 columns per step: two TMEM loads, one wait; then one fp16 box or
+      // two fp32 boxes (staging buffer cb & 3, four boxes in flight)
+      auto put_box = [&](int cb, int col, const uint32_t (&v)[32]) {
         if (warp_full) {
           const uint32_t buf = stage + (cb & 3) * 4096;
           if (cb >= 4) {
@@ -810,6 +781,36 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
                                   : reinterpret_cast<uint4*>(a.o + orow * DC + col);
 #pragma unroll
           for (int q = 0; q < 8; ++q) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      };
+#pragma unroll 1
+      for (int ck = 0; ck < 4; ++ck) {
+        const int col = eh * 256 + ck * 64;
+        uint32_t t0[32], t1[32];
+        if (have_o) {
+          tmem_ld32(tmem + lane_base + col, t0);
+          tmem_ld32(tmem + lane_base + col + 32, t1);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) t0[k] = t1[k] = 0u;
+        }
+        if (p.part_f16) {
+          uint32_t v[32];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            v[k] = pack_f16x2(__uint_as_float(t0[2 * k]) * inv, __uint_as_float(t0[2 * k + 1]) * inv);
+            v[16 + k] = pack_f16x2(__uint_as_float(t1[2 * k]) * inv, __uint_as_float(t1[2 * k + 1]) * inv);
+          }
+          put_box(ck, col, v);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            t0[k] = __float_as_uint(__uint_as_float(t0[k]) * inv);
+            t1[k] = __float_as_uint(__uint_as_float(t1[k]) * inv);
+          }
+          put_box(2 * ck, col, t0);
+          put_box(2 * ck + 1, col + 32, t1);
         }
       }
       if (warp_full && lane == 0) bulk_wait_group_read<0>();
