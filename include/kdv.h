@@ -112,7 +112,8 @@ KDV_API const char* kdv_status_string(kdv_status s);
  * kdv_tree_build, kdv_absorb_q / kdv_unabsorb_o and KDV_IMPL_TC_STAGED to
  * the 100 set (mask build, verify, no-alloc verify, combine); 120 adds
  * kdv_latent_f16, the wait_limit_ns and v16 fields of kdv_verify_params,
- * KDV_DERR_RANGE, and retires KDV_IMPL_TC_1SM. */
+ * KDV_DERR_RANGE, and retires KDV_IMPL_TC_1SM; 121 adds kdv_absorb_q_ex /
+ * kdv_unabsorb_o_ex. */
 KDV_API int32_t kdv_version(void);
 
 /*
@@ -363,6 +364,26 @@ KDV_API kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_laten
 KDV_API kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v,
                                   const float* o_lat, int64_t o_lat_stride, const void* w_uv, int32_t w_dtype,
                                   void* out, int64_t out_stride, int32_t out_dtype, void* stream);
+
+/*
+ * kdv_absorb_q_ex / kdv_unabsorb_o_ex -- the same, with flags (0 = the calls
+ * above). KDV_PROJ_STATIC_WEIGHTS promises that the weights are not written
+ * by the kernel launched immediately before on `stream` (weights of a loaded
+ * model are constant over the step). The TMA-staged kernels are then launched
+ * as programmatic dependents of that kernel: their CTAs start copying weight
+ * tiles while it finishes, and wait for it (griddepcontrol.wait) before they
+ * read q_nope / o_lat or write any output, so every other stream-order
+ * guarantee holds. The general kernels ignore the flag. Unknown flag bits:
+ * KDV_ERR_INVALID_ARG.
+ */
+#define KDV_PROJ_STATIC_WEIGHTS 1u
+KDV_API kdv_status kdv_absorb_q_ex(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope,
+                                   const void* q_nope, int64_t q_nope_stride, int32_t q_dtype, const void* w_uk,
+                                   int32_t w_dtype, void* q_lat, int64_t q_lat_stride, int32_t out_dtype,
+                                   uint32_t flags, void* stream);
+KDV_API kdv_status kdv_unabsorb_o_ex(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v,
+                                     const float* o_lat, int64_t o_lat_stride, const void* w_uv, int32_t w_dtype,
+                                     void* out, int64_t out_stride, int32_t out_dtype, uint32_t flags, void* stream);
 
 /*
  * kdv_tree_build -- best-first draft-tree construction on the device (the

@@ -28,12 +28,14 @@ namespace kdv {
 // absorb_tc.cu: the tensor-core forms (bf16 weights; see the conditions below)
 size_t absorb_tc_smem(int D_n);
 size_t unabsorb_tc_smem(int D_c);
+// early_weights: launch as a programmatic dependent of the preceding kernel
+// (the weight copy may start before that kernel finishes)
 cudaError_t launch_absorb_q_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_n,
                                const void* q_nope, int64_t q_stride, void* q_lat, int64_t o_stride, int32_t o_dtype,
-                               cudaStream_t s);
+                               bool early_weights, cudaStream_t s);
 cudaError_t launch_unabsorb_o_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_v,
                                  const float* o_lat, int64_t i_stride, void* out, int64_t o_stride, int32_t o_dtype,
-                                 cudaStream_t s);
+                                 bool early_weights, cudaStream_t s);
 
 namespace {
 
@@ -556,9 +558,10 @@ using namespace kdv;
 
 extern "C" {
 
-kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope, const void* q_nope,
-                        int64_t q_nope_stride, int32_t q_dtype, const void* w_uk, int32_t w_dtype, void* q_lat,
-                        int64_t q_lat_stride, int32_t out_dtype, void* stream) {
+kdv_status kdv_absorb_q_ex(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope, const void* q_nope,
+                           int64_t q_nope_stride, int32_t q_dtype, const void* w_uk, int32_t w_dtype, void* q_lat,
+                           int64_t q_lat_stride, int32_t out_dtype, uint32_t flags, void* stream) {
+  if ((flags & ~KDV_PROJ_STATIC_WEIGHTS) != 0) return KDV_ERR_INVALID_ARG;
   kdv_status st = check_common(rows, num_heads, d_nope, d_latent, q_nope, q_nope_stride, w_uk, w_dtype, q_lat,
                                q_lat_stride, out_dtype);
   if (st != KDV_OK) return st;
@@ -590,7 +593,8 @@ kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32
       weight_map(&tmap, w_uk, (uint64_t)num_heads * d_latent, (uint64_t)d_nope, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return launch_absorb_q_tc(tmap, rows, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_lat, q_lat_stride,
-                              out_dtype, s) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+                              out_dtype, (flags & KDV_PROJ_STATIC_WEIGHTS) != 0, s) == cudaSuccess ? KDV_OK
+                                                                                                  : KDV_ERR_CUDA;
   if (vec && (int64_t)num_heads * d_latent <= 0x7fffffff &&
       weight_map(&tmap, w_uk, (uint64_t)num_heads * d_latent, (uint64_t)d_nope, 64, PA_ROWS,
                  CU_TENSOR_MAP_SWIZZLE_128B)) {
@@ -612,9 +616,17 @@ kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32
   return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
 }
 
-kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v, const float* o_lat,
-                          int64_t o_lat_stride, const void* w_uv, int32_t w_dtype, void* out, int64_t out_stride,
-                          int32_t out_dtype, void* stream) {
+kdv_status kdv_absorb_q(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_nope, const void* q_nope,
+                        int64_t q_nope_stride, int32_t q_dtype, const void* w_uk, int32_t w_dtype, void* q_lat,
+                        int64_t q_lat_stride, int32_t out_dtype, void* stream) {
+  return kdv_absorb_q_ex(rows, num_heads, d_latent, d_nope, q_nope, q_nope_stride, q_dtype, w_uk, w_dtype, q_lat,
+                         q_lat_stride, out_dtype, 0u, stream);
+}
+
+kdv_status kdv_unabsorb_o_ex(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v, const float* o_lat,
+                             int64_t o_lat_stride, const void* w_uv, int32_t w_dtype, void* out, int64_t out_stride,
+                             int32_t out_dtype, uint32_t flags, void* stream) {
+  if ((flags & ~KDV_PROJ_STATIC_WEIGHTS) != 0) return KDV_ERR_INVALID_ARG;
   kdv_status st = check_common(rows, num_heads, d_latent, d_v, o_lat, o_lat_stride, w_uv, w_dtype, out,
                                out_stride, out_dtype);
   if (st != KDV_OK) return st;
@@ -644,7 +656,7 @@ kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int
       o_lat_stride % 4 == 0 && (int64_t)num_heads * d_latent <= 0x7fffffff &&
       weight_map(&tmap, w_uv, (uint64_t)num_heads * d_latent, (uint64_t)d_v, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return launch_unabsorb_o_tc(tmap, rows, num_heads, d_latent, d_v, o_lat, o_lat_stride, out, out_stride, out_dtype,
-                                s) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+                                (flags & KDV_PROJ_STATIC_WEIGHTS) != 0, s) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
   if (w_dtype == KDV_BF16 && d_v % 8 == 0 && d_latent <= PU_MAX_DC &&
       (reinterpret_cast<uintptr_t>(w_uv) & 15) == 0 && (int64_t)num_heads * d_latent <= 0x7fffffff &&
       weight_map(&tmap, w_uv, (uint64_t)num_heads * d_latent, (uint64_t)d_v, PU_V, 256,
@@ -664,6 +676,13 @@ kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int
     unabsorb_o_kernel<false><<<grid, U_THREADS, smem, s>>>(rows / num_heads, num_heads, d_latent, d_v, o_lat,
                                                            o_lat_stride, w_uv, w_dtype, out, out_stride, out_dtype);
   return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+}
+
+kdv_status kdv_unabsorb_o(int32_t rows, int32_t num_heads, int32_t d_latent, int32_t d_v, const float* o_lat,
+                          int64_t o_lat_stride, const void* w_uv, int32_t w_dtype, void* out, int64_t out_stride,
+                          int32_t out_dtype, void* stream) {
+  return kdv_unabsorb_o_ex(rows, num_heads, d_latent, d_v, o_lat, o_lat_stride, w_uv, w_dtype, out, out_stride,
+                           out_dtype, 0u, stream);
 }
 
 }  // extern "C"

@@ -27,6 +27,12 @@
 // Every wait is bounded (2 s); a CTA whose weights or MMAs never complete
 // writes NaN to its outputs instead of waiting forever (these entry points
 // take no device error flag).
+//
+// Launched as a programmatic dependent (the caller's "static weights" flag),
+// a CTA starts its weight copy before the preceding kernel on the stream has
+// finished and waits for that kernel (griddepcontrol.wait) only before it
+// reads q_nope / o_lat or writes anything; launched normally the wait is a
+// no-op. Each CTA also lets the next such launch begin at once.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -115,6 +121,8 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per_
     tmem_alloc(smem_u32(&tmem_slot), tmem_cols_for(A_MAXN));
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -191,6 +199,8 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
     tmem_alloc(smem_u32(&tmem_slot), tmem_cols_for(U_MAXN));
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -259,9 +269,30 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
 size_t absorb_tc_smem(int D_n) { return 1024 + (size_t)(D_n / 64) * (BOX + A_MAXN * 128); }
 size_t unabsorb_tc_smem(int D_c) { return 1024 + (size_t)(D_c / 64) * (BOX + 2 * U_MAXN * 128); }
 
+// Launch `kernel` with the programmatic-dependent attribute when `early`.
+template <typename... Args>
+static cudaError_t launch_maybe_early(bool early, void (*kernel)(Args...), dim3 grid, size_t smem, cudaStream_t s,
+                                      Args... args) {
+  if (!early) {
+    kernel<<<grid, TC_THREADS, smem, s>>>(args...);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t launch_absorb_q_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_n,
                                const void* q_nope, int64_t q_stride, void* q_lat, int64_t o_stride, int32_t o_dtype,
-                               cudaStream_t s) {
+                               bool early_weights, cudaStream_t s) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -272,14 +303,13 @@ cudaError_t launch_absorb_q_tc(const CUtensorMap& tmap, int32_t rows, int32_t H,
     attr_set[dev] = true;
   }
   const dim3 grid((unsigned)(D_c / 128), (unsigned)H);
-  absorb_q_tc_kernel<<<grid, TC_THREADS, absorb_tc_smem(D_n), s>>>(
-      tmap, rows / H, H, D_c, D_n, static_cast<const __nv_bfloat16*>(q_nope), q_stride, q_lat, o_stride, o_dtype);
-  return cudaGetLastError();
+  return launch_maybe_early(early_weights, absorb_q_tc_kernel, grid, absorb_tc_smem(D_n), s, tmap, rows / H, H, D_c,
+                            D_n, static_cast<const __nv_bfloat16*>(q_nope), q_stride, q_lat, o_stride, (int)o_dtype);
 }
 
 cudaError_t launch_unabsorb_o_tc(const CUtensorMap& tmap, int32_t rows, int32_t H, int32_t D_c, int32_t D_v,
                                  const float* o_lat, int64_t i_stride, void* out, int64_t o_stride, int32_t o_dtype,
-                                 cudaStream_t s) {
+                                 bool early_weights, cudaStream_t s) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -291,9 +321,8 @@ cudaError_t launch_unabsorb_o_tc(const CUtensorMap& tmap, int32_t rows, int32_t 
     attr_set[dev] = true;
   }
   const dim3 grid((unsigned)(D_v / 128), (unsigned)H);
-  unabsorb_o_tc_kernel<<<grid, TC_THREADS, unabsorb_tc_smem(D_c), s>>>(tmap, rows / H, H, D_c, D_v, o_lat, i_stride,
-                                                                       out, o_stride, o_dtype);
-  return cudaGetLastError();
+  return launch_maybe_early(early_weights, unabsorb_o_tc_kernel, grid, unabsorb_tc_smem(D_c), s, tmap, rows / H, H,
+                            D_c, D_v, o_lat, i_stride, out, o_stride, (int)o_dtype);
 }
 
 }  // namespace kdv

@@ -275,7 +275,7 @@ const char* kdv_status_string(kdv_status s) {
   return "KDV_ERR_UNKNOWN";
 }
 
-int32_t kdv_version(void) { return 120; }
+int32_t kdv_version(void) { return 121; }
 
 kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
                                int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,

@@ -34,6 +34,7 @@ KDV_DERR_RANGE = 7
 
 KDV_BF16 = 0
 KDV_F32 = 1
+KDV_PROJ_STATIC_WEIGHTS = 1     # kdv_absorb_q_ex / kdv_unabsorb_o_ex flag: weights not written by the previous kernel
 KDV_IMPL_AUTO = 0
 KDV_IMPL_SIMT = 1
 KDV_IMPL_TC = 2
@@ -46,7 +47,8 @@ KDV_MAX_BATCH = 128
 EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
             "kdv_verify_attn_noalloc", "kdv_latent_f16", "kdv_combine", "kdv_tree_accept_workspace",
-            "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o", "kdv_tree_build")
+            "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o", "kdv_tree_build",
+            "kdv_absorb_q_ex", "kdv_unabsorb_o_ex")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -148,6 +150,10 @@ def load() -> ctypes.CDLL:
         lib.kdv_unabsorb_o.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int32, c.c_void_p, c.c_int64,
                                        c.c_void_p, c.c_int32, c.c_void_p, c.c_int64, c.c_int32, c.c_void_p]
         lib.kdv_unabsorb_o.restype = c.c_int
+        lib.kdv_absorb_q_ex.argtypes = list(lib.kdv_absorb_q.argtypes[:-1]) + [c.c_uint32, c.c_void_p]
+        lib.kdv_absorb_q_ex.restype = c.c_int
+        lib.kdv_unabsorb_o_ex.argtypes = list(lib.kdv_unabsorb_o.argtypes[:-1]) + [c.c_uint32, c.c_void_p]
+        lib.kdv_unabsorb_o_ex.restype = c.c_int
         lib.kdv_tree_build.argtypes = [c.POINTER(BuildParams), c.c_void_p]
         lib.kdv_tree_build.restype = c.c_int
         _lib = lib
@@ -251,23 +257,31 @@ def _dt(t: torch.Tensor) -> int:
 
 
 def kdv_absorb_q(num_heads: int, q_nope: torch.Tensor, w_uk: torch.Tensor, q_lat: torch.Tensor,
-                 stream=None) -> None:
-    """q_lat[row, :D_c] = W_UK[row % H] q_nope[row] (2-D row-strided tensors)."""
+                 stream=None, flags: int = 0) -> None:
+    """q_lat[row, :D_c] = W_UK[row % H] q_nope[row] (2-D row-strided tensors).
+    flags != 0 calls kdv_absorb_q_ex (KDV_PROJ_STATIC_WEIGHTS)."""
     rows, d_nope = q_nope.shape
     d_latent = w_uk.shape[1]
-    _check(load().kdv_absorb_q(int(rows), int(num_heads), int(d_latent), int(d_nope), _ptr(q_nope),
-                               int(q_nope.stride(0)), _dt(q_nope), _ptr(w_uk), _dt(w_uk), _ptr(q_lat),
-                               int(q_lat.stride(0)), _dt(q_lat), _stream(stream)), "kdv_absorb_q")
+    args = (int(rows), int(num_heads), int(d_latent), int(d_nope), _ptr(q_nope), int(q_nope.stride(0)),
+            _dt(q_nope), _ptr(w_uk), _dt(w_uk), _ptr(q_lat), int(q_lat.stride(0)), _dt(q_lat))
+    if flags:
+        _check(load().kdv_absorb_q_ex(*args, int(flags), _stream(stream)), "kdv_absorb_q_ex")
+    else:
+        _check(load().kdv_absorb_q(*args, _stream(stream)), "kdv_absorb_q")
 
 
 def kdv_unabsorb_o(num_heads: int, o_lat: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor,
-                   stream=None) -> None:
-    """out[row] = W_UV[row % H]^T o_lat[row] (o_lat fp32)."""
+                   stream=None, flags: int = 0) -> None:
+    """out[row] = W_UV[row % H]^T o_lat[row] (o_lat fp32).
+    flags != 0 calls kdv_unabsorb_o_ex (KDV_PROJ_STATIC_WEIGHTS)."""
     rows, d_latent = o_lat.shape
     d_v = w_uv.shape[2]
-    _check(load().kdv_unabsorb_o(int(rows), int(num_heads), int(d_latent), int(d_v), _ptr(o_lat),
-                                 int(o_lat.stride(0)), _ptr(w_uv), _dt(w_uv), _ptr(out), int(out.stride(0)),
-                                 _dt(out), _stream(stream)), "kdv_unabsorb_o")
+    args = (int(rows), int(num_heads), int(d_latent), int(d_v), _ptr(o_lat), int(o_lat.stride(0)), _ptr(w_uv),
+            _dt(w_uv), _ptr(out), int(out.stride(0)), _dt(out))
+    if flags:
+        _check(load().kdv_unabsorb_o_ex(*args, int(flags), _stream(stream)), "kdv_unabsorb_o_ex")
+    else:
+        _check(load().kdv_unabsorb_o(*args, _stream(stream)), "kdv_unabsorb_o")
 
 
 def kdv_combine(o_part: torch.Tensor, lse_part: torch.Tensor, S: int, rows: int, d: int,

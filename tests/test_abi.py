@@ -38,7 +38,7 @@ def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4):
         assert kdv.status_string(s).startswith("KDV_")
     assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
-    assert kdv.kdv_version() == 120
+    assert kdv.kdv_version() == 121
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
@@ -227,6 +227,14 @@ def test_projection_validation(lib):
     assert fu(13, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_INVALID_ARG
     assert fu(16, 4, 513, 128, 0x1000, 513, 0x2000, B, 0x3000, 128, F, None) == kdv.KDV_ERR_UNSUPPORTED
     assert fu(16, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 100, F, None) == kdv.KDV_ERR_INVALID_ARG
+    # the flagged forms validate the same way and refuse unknown flag bits
+    fax, fux = lib.kdv_absorb_q_ex, lib.kdv_unabsorb_o_ex
+    S = kdv.KDV_PROJ_STATIC_WEIGHTS
+    assert fax(13, 4, 512, 128, 0x1000, 128, B, 0x2000, B, 0x3000, 576, B, S, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fax(0, 4, 512, 128, None, 128, B, None, B, None, 576, B, S, None) == kdv.KDV_OK
+    assert fax(0, 4, 512, 128, None, 128, B, None, B, None, 576, B, 2, None) == kdv.KDV_ERR_INVALID_ARG
+    assert fux(16, 4, 513, 128, 0x1000, 513, 0x2000, B, 0x3000, 128, F, S, None) == kdv.KDV_ERR_UNSUPPORTED
+    assert fux(16, 4, 512, 128, 0x1000, 512, 0x2000, B, 0x3000, 128, F, 4, None) == kdv.KDV_ERR_INVALID_ARG
 
 
 def test_tree_build_validation(lib):

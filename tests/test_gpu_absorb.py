@@ -168,3 +168,30 @@ def test_kimi_layer_end_to_end_bf16():
     assert st["rel_max"] <= floor["rel_max"] + REL_MAX_TOL, (st, floor)
     assert st["rel_mean"] <= floor["rel_mean"] + REL_MEAN_TOL, (st, floor)
     assert st["lse"] <= floor["lse"] + LSE_TOL, (st, floor)
+
+
+@pytest.mark.parametrize("T", [13, 70])
+def test_static_weights_flag_gives_the_same_bits(T):
+    """KDV_PROJ_STATIC_WEIGHTS only changes when the weight copies may start
+    (programmatic dependent launch), not what is computed: a chain of flagged
+    calls -- each a dependent of the one before, the outputs of one call the
+    inputs of the next -- must give the plain calls' bits."""
+    case = datagen.kimi_layer_case(L=64, T=T, seed=7)
+    q_nope, w_uk, w_uv = datagen.layer_weights(case)
+    qn, wk, wv = _t(q_nope, torch.bfloat16), _t(w_uk, torch.bfloat16), _t(w_uv, torch.bfloat16)
+    outs = []
+    for flags in (0, kdv.KDV_PROJ_STATIC_WEIGHTS):
+        q = torch.zeros(case.rows, 576, dtype=torch.bfloat16, device=dev)
+        o_lat = torch.empty(case.rows, 512, device=dev)
+        out = torch.empty(case.rows, 128, device=dev)
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                kdv.kdv_absorb_q(case.H, qn, wk, q[:, :512], s, flags=flags)
+                o_lat.copy_(q[:, :512].float() * 0.01)          # a kernel between that reads the output
+                kdv.kdv_unabsorb_o(case.H, o_lat, wv, out, s, flags=flags)
+                kdv.kdv_unabsorb_o(case.H, o_lat, wv, out, s, flags=flags)   # back to back
+        s.synchronize()
+        outs.append((q.cpu(), out.cpu()))
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    assert torch.equal(outs[0][1].view(torch.int32), outs[1][1].view(torch.int32))
