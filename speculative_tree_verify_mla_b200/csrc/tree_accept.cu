@@ -15,7 +15,9 @@
 //       whether its root path is accepted (each node walks its own ancestors,
 //       so no node waits on another), takes the deepest accepted node (lowest
 //       index on ties), writes the path, the bonus token and optionally
-//       commits the page table in place.
+//       commits the page table in place. It is launched as a programmatic
+//       dependent of the argmax pass (its launch overlaps that pass) and
+//       reads nothing before the pass has finished.
 #include <cuda_runtime.h>
 
 #include "kdv.h"
@@ -49,6 +51,8 @@ __global__ void __launch_bounds__(ARGMAX_THREADS)
 argmax_partial_kernel(const void* __restrict__ logits, int64_t ld, int32_t vocab, int32_t chunks,
                       int vec, unsigned long long* __restrict__ part) {
   const int row = blockIdx.y, chunk = blockIdx.x;
+  // the acceptance kernel may launch now; it waits for this grid to finish
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t c0 = (int64_t)chunk * CHUNK;
   const int64_t c1 = c0 + CHUNK < vocab ? c0 + CHUNK : vocab;
   unsigned long long best = 0ull;
@@ -152,6 +156,10 @@ __global__ void __launch_bounds__(ACCEPT_THREADS) accept_tree_kernel(const Accep
   __shared__ int32_t s_path[MAX_NODES];
   __shared__ unsigned long long s_key[ACCEPT_THREADS / 32];
   __shared__ int s_off_count;
+  // launched as a programmatic dependent of the argmax pass: nothing is read
+  // before that grid (and so all earlier work on the stream) has finished;
+  // a no-op when launched normally
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int t0 = a.tree_off[b];
   const int T = a.tree_off[b + 1] - t0;
@@ -335,8 +343,21 @@ kdv_status kdv_tree_accept(const kdv_accept_params* p, void* stream) {
     if (cudaGetLastError() != cudaSuccess) return KDV_ERR_CUDA;
     a.part = part;
   }
-  accept_tree_kernel<<<p->batch, ACCEPT_THREADS, 0, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+  if (p->logits == nullptr) {
+    accept_tree_kernel<<<p->batch, ACCEPT_THREADS, 0, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
+  }
+  // right behind the argmax pass: launch as its programmatic dependent
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p->batch);
+  cfg.blockDim = dim3(ACCEPT_THREADS);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, accept_tree_kernel, a) == cudaSuccess ? KDV_OK : KDV_ERR_CUDA;
 }
 
 }  // extern "C"
