@@ -131,13 +131,26 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_per_
   int pass = 0;
   for (int t0 = 0; t0 < rows_per_head; t0 += A_MAXN, ++pass) {
     const int n = min(A_MAXN, rows_per_head - t0), npad = (n + 15) & ~15;
-    // B: node t's D_n dims as nkb swizzled rows of 128 bytes (zeros past n)
-    for (int i = threadIdx.x; i < npad * nkb * 8; i += TC_THREADS) {
-      const int ch = i & 7, kb = (i >> 3) % nkb, t = (i >> 3) / nkb;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t < n)
-        v = *reinterpret_cast<const uint4*>(q_nope + ((int64_t)(t0 + t) * H + h) * q_stride + kb * 64 + ch * 8);
-      st_shared_v4(s_b + kb * (A_MAXN * 128) + t * 128 + ((ch ^ (t & 7)) << 4), v.x, v.y, v.z, v.w);
+    // B: node t's D_n dims as nkb swizzled rows of 128 bytes (zeros past
+    // n); four items' loads go out before any (ordered) shared store
+    const int total = npad * nkb * 8;
+    for (int i0 = threadIdx.x; i0 < total; i0 += 4 * TC_THREADS) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * TC_THREADS;
+        const int ch = i & 7, kb = (i >> 3) % nkb, t = (i >> 3) / nkb;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < total && t < n)
+          v[u] = *reinterpret_cast<const uint4*>(q_nope + ((int64_t)(t0 + t) * H + h) * q_stride + kb * 64 + ch * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * TC_THREADS;
+        if (i >= total) break;
+        const int ch = i & 7, kb = (i >> 3) % nkb, t = (i >> 3) / nkb;
+        st_shared_v4(s_b + kb * (A_MAXN * 128) + t * 128 + ((ch ^ (t & 7)) << 4), v[u].x, v[u].y, v[u].z, v[u].w);
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -209,15 +222,30 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
   int pass = 0;
   for (int t0 = 0; t0 < rows_per_head; t0 += U_MAXN, ++pass) {
     const int n = min(U_MAXN, rows_per_head - t0), npad = (n + 15) & ~15;
-    // B: node t's D_c values as bf16 hi and lo parts, swizzled 128-byte rows
-    for (int i = threadIdx.x; i < npad * ncb * 8; i += TC_THREADS) {
-      const int ch = i & 7, cb = (i >> 3) % ncb, t = (i >> 3) / ncb;
-      uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-      if (t < n) {
-        const float* src = o_lat + ((int64_t)(t0 + t) * H + h) * i_stride + cb * 64 + ch * 8;
-        const float4 a = *reinterpret_cast<const float4*>(src);
-        const float4 b = *reinterpret_cast<const float4*>(src + 4);
-        const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    // B: node t's D_c values as bf16 hi and lo parts, swizzled 128-byte
+    // rows. Four items' loads go out before any store (the shared stores
+    // are ordered asm, so a load after one would wait for it).
+    const int total = npad * ncb * 8;
+    for (int i0 = threadIdx.x; i0 < total; i0 += 4 * TC_THREADS) {
+      float4 xa[4], xb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * TC_THREADS;
+        const int ch = i & 7, cb = (i >> 3) % ncb, t = (i >> 3) / ncb;
+        xa[u] = xb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < total && t < n) {
+          const float* src = o_lat + ((int64_t)(t0 + t) * H + h) * i_stride + cb * 64 + ch * 8;
+          xa[u] = *reinterpret_cast<const float4*>(src);
+          xb[u] = *reinterpret_cast<const float4*>(src + 4);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * TC_THREADS;
+        if (i >= total) break;
+        const int ch = i & 7, cb = (i >> 3) % ncb, t = (i >> 3) / ncb;
+        const float x[8] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w, xb[u].x, xb[u].y, xb[u].z, xb[u].w};
+        uint32_t hi[4], lo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * j]), h1 = __float2bfloat16_rn(x[2 * j + 1]);
@@ -226,10 +254,10 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
           hi[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
           lo[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
         }
+        const uint32_t off = cb * BB + t * 128 + ((ch ^ (t & 7)) << 4);
+        st_shared_v4(s_hi + off, hi[0], hi[1], hi[2], hi[3]);
+        st_shared_v4(s_lo + off, lo[0], lo[1], lo[2], lo[3]);
       }
-      const uint32_t off = cb * BB + t * 128 + ((ch ^ (t & 7)) << 4);
-      st_shared_v4(s_hi + off, hi[0], hi[1], hi[2], hi[3]);
-      st_shared_v4(s_lo + off, lo[0], lo[1], lo[2], lo[3]);
     }
     fence_proxy_async_smem();
     __syncthreads();
