@@ -223,13 +223,13 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
   for (int t0 = 0; t0 < rows_per_head; t0 += U_MAXN, ++pass) {
     const int n = min(U_MAXN, rows_per_head - t0), npad = (n + 15) & ~15;
     // B: node t's D_c values as bf16 hi and lo parts, swizzled 128-byte
-    // rows. Four items' loads go out before any store (the shared stores
+    // rows. Eight items' loads go out before any store (the shared stores
     // are ordered asm, so a load after one would wait for it).
     const int total = npad * ncb * 8;
-    for (int i0 = threadIdx.x; i0 < total; i0 += 4 * TC_THREADS) {
-      float4 xa[4], xb[4];
+    for (int i0 = threadIdx.x; i0 < total; i0 += 8 * TC_THREADS) {
+      float4 xa[8], xb[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * TC_THREADS;
         const int ch = i & 7, cb = (i >> 3) % ncb, t = (i >> 3) / ncb;
         xa[u] = xb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -240,7 +240,7 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * TC_THREADS;
         if (i >= total) break;
         const int ch = i & 7, cb = (i >> 3) % ncb, t = (i >> 3) / ncb;
