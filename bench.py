@@ -13,9 +13,10 @@ graph of the step; the metric is microseconds per layer.
 
 Also reported: the dominant kernel's roofline (tensor bound), an end-to-end
 number through the C ABI with host buffers, the CPU oracle as a baseline, and
-sub-records for the other configurations -- the 200k-key long context and
-the 8-request paged batch, each with its own roofline -- plus greedy
-acceptance, the two projections and the tree builder.
+sub-records for the other configurations -- the 200k-key long context, the
+8-request paged batch and the context sweep (L = 13, 1663, 3333, 5553), each
+with its own roofline -- plus greedy acceptance, the two projections and the
+tree builder.
 
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
 torchrun, each rank runs its own layers (weak scaling, no collective on the
@@ -543,6 +544,30 @@ def time_config(name: str, dev, stream, peaks, impl_code: int = 0, reps: int = 2
             "timing": f"CUDA graph of one call, {reps} replays, CUDA events on the launch stream"}
 
 
+def time_sweep(dev, stream, peaks, n_layers: int = 61, reps: int = 5):
+    """The context sweep (T=15, 61 distinct layers per step) at every swept
+    prefix length: µs per layer of the whole step from a CUDA graph replay,
+    against that layer's roofline."""
+    import torch
+    res = {"workload": "context_sweep_T15", "layers_per_step": n_layers,
+           "timing": f"CUDA graph of the {n_layers}-layer step, {reps} replays"}
+    for L in SWEEP_L:
+        prob = Problems(workload_cases("sweep", n_layers, L=L), 0, dev)
+        with torch.cuda.stream(stream):
+            prob.step(stream)
+        stream.synchronize()
+        g = graph_of(prob.step, stream)
+        us = replay_us(g, stream, reps) / n_layers
+        del g
+        flops, kv_bytes = case_flops_bytes(prob.cases[0])
+        roof_us = max(flops / (peaks["bf16_tflops"] * 1e12), kv_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+        res[f"L{L}"] = {"us_per_layer": us, "roofline_us": roof_us, "frac_of_roofline": roof_us / us,
+                        "splits": prob.splits[0], "d_err": int(prob.d_err.item())}
+        del prob
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args):
     import torch
     from speculative_tree_verify_mla_b200 import kdv
@@ -718,6 +743,7 @@ def run_gpu(args):
     if args.workload == "kimi" and rank == 0 and not args.headline_only:
         result["long_context"] = time_config("long", dev, stream, peaks)
         result["paged"] = time_config("paged", dev, stream, peaks)
+        result["context_sweep"] = time_sweep(dev, stream, peaks)
         result["tree_accept"] = time_tree_accept(dev, stream, peaks)
         result["projections"] = time_projections(dev, stream, peaks)
         result["tree_build"] = time_tree_build(dev, stream)
