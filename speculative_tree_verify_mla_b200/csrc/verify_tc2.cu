@@ -23,22 +23,26 @@
 //     the next tile's rows are prefetched into L2 meanwhile. TMEM holds two
 //     S buffers of 256 columns, so the MMAs of tile i+1 (issued by CTA 0)
 //     run while the softmax warps drain tile i. Two softmax warpgroups per
-//     CTA (one row per thread, keys 0-127 and 128-255 of the tile) share the
-//     row maximum through shared memory, and each pushes its fp16 P half to
-//     the partner CTA on the O side with st.async.
+//     CTA (one row per thread, keys 0-127 and 128-255 of the tile) agree on
+//     the row maximum (a barrier vote; an exchange through shared memory
+//     only when some row's reference max may move), and each pushes its fp16
+//     P half to the partner CTA on the O side with st.async, the second
+//     warpgroup half a P tile behind the first so that one's exp2 work
+//     overlaps the other's pushes.
 //   CTA 2 + CTA 3 ("O pair"): O += P V with M=256, N=256 (two MMAs per 16
 //     keys), K=16, per 128-key P tile. O (128 rows x 512 fp32) fills each
 //     CTA's TMEM; each CTA stages 256 of the 512 V dims (the half of each
-//     N=256 column range the MMA expects from it) through a 16 KB x 6 ring,
-//     with TMA boxes from the call's fp16 copy of the latent rows (below).
-//     CTA 2 issues the MMAs.
+//     N=256 column range the MMA expects from it) through a 16 KB x 5 ring,
+//     with TMA boxes from the call's fp16 copy of the latent rows (below),
+//     and takes P tiles into 4 slots. CTA 2 issues the MMAs.
 //
 // Precision of P.V. The softmax numerators P are rounded to a 16-bit type
 // before the P.V MMA, and that rounding is the kernel's dominant error. In
 // bf16 (8 significant bits) it leaves a normalised mean error near 1e-3 of
 // the output's RMS; in fp16 (11 bits) about 1.3e-4. A kind::f16 MMA takes A
 // and B of one type, so V is read as fp16 too, from rows that
-// latent_f16.cu writes before this kernel runs (bf16 -> fp16 is exact for
+// latent_f16.cu writes before this kernel (which may be launched as that
+// pass's programmatic dependent; only the V loads wait for it) (bf16 -> fp16 is exact for
 // every latent value with 2^-14 <= |x| < 65536). V cannot be converted here:
 // while the tensor core streams shared memory the load/store unit gets only
 // ~5-10 B/clk of it (measured), so reading a 16 KB stage back through
