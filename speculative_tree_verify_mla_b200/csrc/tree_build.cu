@@ -11,8 +11,9 @@
 // log-probabilities <= 0 that is the first T nodes of that order.
 //
 // One warp per request, no block barrier anywhere. Frontier entry i belongs
-// to lane i % 32, which alone writes and reads its fields in shared memory;
-// every lane keeps the best of its own live entries in registers. A round is
+// to lane i % 32: its score image and path key live in that lane's registers
+// (stripe i / 32), its depth, parent and token in shared memory, and every
+// lane keeps the best of its own live entries. A round is
 // then a warp-wide selection of the best lane-best under that total order
 // (redux max over an order-preserving integer image of the score, redux min
 // over the unique path key only when scores tie), after which the winner's
@@ -71,10 +72,16 @@ __device__ __forceinline__ bool before(uint32_t ia, unsigned long long ka, uint3
 }
 
 __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildArgs a) {
-  // frontier entries; entry i is touched by lane i % 32 only
-  __shared__ uint32_t e_img[MAX_FRONTIER];
-  __shared__ unsigned long long e_key[MAX_FRONTIER];
+  // frontier entries; entry i is touched by lane i % 32 only: score image
+  // and path key in that lane's registers (stripe i / 32), the rest here
   __shared__ int32_t e_depth[MAX_FRONTIER], e_parent[MAX_FRONTIER], e_token[MAX_FRONTIER];
+  uint32_t r_img[NSTRIPE];
+  unsigned long long r_key[NSTRIPE];
+#pragma unroll
+  for (int st = 0; st < NSTRIPE; ++st) {
+    r_img[st] = 0u;
+    r_key[st] = 0ull;
+  }
   __shared__ float s_logp[MAX_D * MAX_K];
   __shared__ int32_t s_tok[MAX_D * MAX_K];
   __shared__ unsigned long long s_place[MAX_D + 1];
@@ -121,8 +128,8 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
   unsigned long long lb_key = 0ull;
   int lb_dep = 0, lb_idx = -1;
   if (lane == 0) {
-    e_img[0] = score_img(0.f);
-    e_key[0] = 0ull;
+    r_img[0] = score_img(0.f);
+    r_key[0] = 0ull;
     e_depth[0] = 0;
     e_parent[0] = -1;
     e_token[0] = a.root_token[b];
@@ -157,24 +164,25 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
       a.token[t0 + n] = e_token[bi];
       if (a.depth) a.depth[t0 + n] = dep;
       if (a.score) a.score[t0 + n] = bs;
-      e_img[bi] = 0u;
+      const int bst = bi / BUILD_THREADS;
       uint32_t c_img[NSTRIPE];
       unsigned long long c_key[NSTRIPE];
       int c_st[NSTRIPE];
 #pragma unroll
       for (int st = 0; st < NSTRIPE; ++st) {
-        const int i = lane + st * BUILD_THREADS;
-        const bool have = i < n_front;
-        c_img[st] = have ? e_img[i] : 0u;
-        c_key[st] = have ? e_key[i] : 0ull;
+        if (st == bst) r_img[st] = 0u;             // retire the emitted entry
+        c_img[st] = r_img[st];
+        c_key[st] = r_key[st];
         c_st[st] = st;
       }
-      // pairwise tournament: 5 levels instead of a 16-long chain
+      // pairwise tournament: 5 levels instead of a 16-long chain, over the
+      // stripes the frontier has reached so far (the bound is warp-uniform)
+      const int nst = (n_front + BUILD_THREADS - 1) / BUILD_THREADS;
 #pragma unroll
       for (int w = 1; w < NSTRIPE; w *= 2) {
 #pragma unroll
         for (int st = 0; st + w < NSTRIPE; st += 2 * w) {
-          if (before(c_img[st + w], c_key[st + w], c_img[st], c_key[st])) {
+          if (st + w < nst && before(c_img[st + w], c_key[st + w], c_img[st], c_key[st])) {
             c_img[st] = c_img[st + w];
             c_key[st] = c_key[st + w];
             c_st[st] = c_st[st + w];
@@ -195,8 +203,13 @@ __global__ void __launch_bounds__(BUILD_THREADS) tree_build_kernel(const BuildAr
         if (isnan(sc)) sc = -INFINITY;             // +inf + -inf: no defined score
         const uint32_t img = score_img(sc);
         const unsigned long long ky = bk + (unsigned long long)(j + 1) * s_place[dep + 1];
-        e_img[i] = img;
-        e_key[i] = ky;
+        const int ist = i / BUILD_THREADS;
+#pragma unroll
+        for (int st = 0; st < NSTRIPE; ++st)
+          if (st == ist) {
+            r_img[st] = img;
+            r_key[st] = ky;
+          }
         e_depth[i] = dep + 1;
         e_parent[i] = n;
         e_token[i] = s_tok[dep * K + j];
