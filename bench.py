@@ -762,7 +762,9 @@ def run_gpu(args):
         "clocks": clocks,
     }
 
-    if args.workload == "kimi" and rank == 0 and not args.headline_only:
+    # single-GPU sub-records: at N=1 only (under torchrun the other ranks
+    # would sit idle in teardown while rank 0 measures them)
+    if args.workload == "kimi" and rank == 0 and world == 1 and not args.headline_only:
         result["long_context"] = time_config("long", dev, stream, peaks)
         result["paged"] = time_config("paged", dev, stream, peaks)
         result["context_sweep"] = time_sweep(dev, stream, peaks)
