@@ -20,7 +20,9 @@ def test_load_peaks_falls_back_when_missing(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
     pk = bench.load_peaks()
     assert pk["source"] == "fallback"
-    assert pk["bf16_tflops"] == pk["bf16_tflops_sustained"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    assert pk["bf16_tflops"] == 1590.0 and pk["hbm_gbs"] == 6650.0
+    # held under the power cap the same GEMM settles lower than its burst rate
+    assert pk["bf16_tflops_sustained"] == 1400.0 < pk["bf16_tflops"]
 
 
 def test_tensor_fracs():
