@@ -299,7 +299,7 @@ class Problems:
         self.trees = {}          # tree bytes -> (parent, tree_off, batch, max_T, mask)
         self.q, self.kv, self.o, self.lse, self.ws, self.params, self.tc_params = [], [], [], [], [], [], []
         self.page_table, self.kv_off, self.tree_off, self.keep = [], [], [], []
-        self.splits, self.items, self.n_combine = [], [], 0
+        self.splits, self.items = [], []
         self.v16, self.n_keys = [], []
         self.tc = impl_code in (kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_STAGED, kdv.KDV_IMPL_AUTO)
         for c in cases:
@@ -326,8 +326,6 @@ class Problems:
             ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
             p.workspace, p.workspace_bytes = ws.data_ptr(), nbytes
             splits, items = kdv.kdv_verify_attn_plan(p)
-            if max(splits) > 1:
-                self.n_combine += 1
             # partials-out twin (uniform S = the largest planned split count)
             S = max(splits)
             o_part = torch.empty(S, c.rows, 512, dtype=torch.float32, device=dev)
@@ -370,8 +368,9 @@ class Problems:
 
     def launches_per_step(self):
         # mask builds, then per call: the fp16 latent rows, the attention
-        # kernel and (with splits) the merge
-        return len(self.trees) + (2 if self.tc else 1) * len(self.params) + self.n_combine
+        # kernel and, unless that kernel merges its own splits, the merge
+        from speculative_tree_verify_mla_b200 import kdv
+        return len(self.trees) + sum(kdv.kdv_verify_attn_launches(p) for p in self.params)
 
 
 def graph_of(fn, stream):

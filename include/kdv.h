@@ -113,7 +113,7 @@ KDV_API const char* kdv_status_string(kdv_status s);
  * the 100 set (mask build, verify, no-alloc verify, combine); 120 adds
  * kdv_latent_f16, the wait_limit_ns and v16 fields of kdv_verify_params,
  * KDV_DERR_RANGE, and retires KDV_IMPL_TC_1SM; 121 adds kdv_absorb_q_ex /
- * kdv_unabsorb_o_ex. */
+ * kdv_unabsorb_o_ex; 122 adds kdv_verify_attn_launches. */
 KDV_API int32_t kdv_version(void);
 
 /*
@@ -205,6 +205,13 @@ KDV_API kdv_status kdv_verify_attn_workspace(const kdv_verify_params* p, size_t*
  * split count. */
 KDV_API kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* splits,
                                         int32_t* grid_items);
+
+/* How many kernels kdv_verify_attn launches for these parameters (host
+ * fields only; writes *launches): the attention kernel, plus the fp16
+ * latent-row pass when the TC kernel writes its own rows (or stages a paged
+ * pool), plus the merge kernel when split partials are merged in the
+ * workspace. For building CUDA graphs and counting launches. */
+KDV_API kdv_status kdv_verify_attn_launches(const kdv_verify_params* p, int32_t* launches);
 
 /*
  * kdv_verify_attn -- tree-verify MLA attention in absorbed form.

@@ -109,10 +109,12 @@ combine_plan_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws
 
 // The internal merge of the tensor-core kernel's fp16 partials (d = 512):
 // one warp per row, lane l owning columns [16l, 16l+16). The loads of the
-// first eight splits are issued before the split LSEs are reduced, so a
-// row with S <= 8 costs about one memory round trip.
+// first eight splits are issued together with those of the split LSEs,
+// which are read once (lane k keeps lse_k), so a row with S <= 8 costs
+// about one memory round trip.
 constexpr int W16_WARPS = 4;
 constexpr int W16_KB = 8;
+constexpr int W16_SMEM = 100 * 1024;   // reserved, unused: two CTAs per SM at most
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -139,6 +141,9 @@ combine_plan_f16_kernel(const __half* __restrict__ ws_o, const float* __restrict
                         const VerifyPlan p, float* __restrict__ o, float* __restrict__ lse) {
   constexpr int D = 512;
   const int lane = threadIdx.x & 31;
+  // launched as a programmatic dependent of the attention kernel: wait for
+  // it to complete (and its partials to be visible)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int64_t row = (int64_t)blockIdx.x * W16_WARPS + (threadIdx.x >> 5); row < p.total_rows;
        row += (int64_t)gridDim.x * W16_WARPS) {
     int b = 0;
@@ -155,8 +160,9 @@ combine_plan_f16_kernel(const __half* __restrict__ ws_o, const float* __restrict
         x[u][0] = __ldg(src);
         x[u][1] = __ldg(src + 1);
       }
-    float m = -INFINITY;
-    for (int k = lane; k < S; k += 32) m = fmaxf(m, __ldg(ws_lse + first + (int64_t)k * rows_b));
+    const float lk0 = lane < S ? __ldg(ws_lse + first + (int64_t)lane * rows_b) : -INFINITY;
+    float m = fmaxf(-INFINITY, lk0);
+    for (int k = lane + 32; k < S; k += 32) m = fmaxf(m, __ldg(ws_lse + first + (int64_t)k * rows_b));
     m = warp_max(m);
     float acc[16];
 #pragma unroll
@@ -164,14 +170,15 @@ combine_plan_f16_kernel(const __half* __restrict__ ws_o, const float* __restrict
     float LSE = -INFINITY;
     if (m != -INFINITY) {
       float z = 0.f;
-      for (int k = lane; k < S; k += 32) {
+      if (lane < S) z += lk0 == -INFINITY ? 0.f : expf(lk0 - m);
+      for (int k = lane + 32; k < S; k += 32) {
         const float lk = __ldg(ws_lse + first + (int64_t)k * rows_b);
         z += lk == -INFINITY ? 0.f : expf(lk - m);
       }
       LSE = m + logf(warp_sum(z));
       for (int k0 = 0; k0 < S; k0 += 32) {
         const int kk = k0 + lane;
-        const float lk = kk < S ? __ldg(ws_lse + first + (int64_t)kk * rows_b) : -INFINITY;
+        const float lk = k0 == 0 ? lk0 : kk < S ? __ldg(ws_lse + first + (int64_t)kk * rows_b) : -INFINITY;
         const float wk = lk == -INFINITY ? 0.f : expf(lk - LSE);
         const int n = min(32, S - k0);
         for (int j = 0; j < n; j += W16_KB) {
@@ -226,9 +233,32 @@ cudaError_t launch_combine_plan(const void* ws_o, const float* ws_lse, const Ver
     if (d != 512) return cudaErrorInvalidValue;
     const int64_t blocks = (p.total_rows + W16_WARPS - 1) / W16_WARPS;
     const int64_t grid = blocks < (int64_t)1 << 30 ? blocks : (int64_t)1 << 30;
-    combine_plan_f16_kernel<<<(unsigned)grid, 32 * W16_WARPS, 0, stream>>>(static_cast<const __half*>(ws_o), ws_lse,
-                                                                            p, o, lse);
-    return cudaGetLastError();
+    // Launched as a programmatic dependent of the attention kernel, whose
+    // CTAs signal it from their epilogue: its CTAs take the SMs the
+    // attention kernel leaves free and wait there, so it starts without a
+    // launch gap. The shared memory it reserves (and does not use) keeps
+    // at most two of its CTAs on an SM, so the early ones do not gather the
+    // whole merge on the few free SMs.
+    static bool smem_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+      e = cudaFuncSetAttribute(combine_plan_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) smem_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(32 * W16_WARPS);
+    cfg.dynamicSmemBytes = W16_SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, combine_plan_f16_kernel, static_cast<const __half*>(ws_o), ws_lse, p, o, lse);
   }
   const int64_t grid = p.total_rows < (int64_t)1 << 30 ? p.total_rows : (int64_t)1 << 30;
   combine_plan_kernel<<<(unsigned)grid, THREADS, 0, stream>>>(static_cast<const float*>(ws_o), ws_lse, p, d, o,

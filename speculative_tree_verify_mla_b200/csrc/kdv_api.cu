@@ -275,7 +275,7 @@ const char* kdv_status_string(kdv_status s) {
   return "KDV_ERR_UNKNOWN";
 }
 
-int32_t kdv_version(void) { return 121; }
+int32_t kdv_version(void) { return 122; }
 
 kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
                                int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
@@ -313,6 +313,22 @@ kdv_status kdv_verify_attn_plan(const kdv_verify_params* p, int32_t* splits, int
   return KDV_OK;
 }
 
+kdv_status kdv_verify_attn_launches(const kdv_verify_params* p, int32_t* launches) {
+  if (p == nullptr || launches == nullptr) return KDV_ERR_INVALID_ARG;
+  const int impl = resolve_impl(p);
+  kdv_status st = check_params(p, impl);
+  if (st != KDV_OK) return st;
+  VerifyPlan plan;
+  size_t bytes = 0;
+  st = make_plan(p, impl, &plan, &bytes);
+  if (st != KDV_OK) return st;
+  int32_t n = 1;                                                   // the attention kernel
+  if ((is_tc2(impl) && p->v16 == nullptr) || staged_paged(p, impl)) ++n;   // the latent pass
+  if (plan.out_mode == OUT_WORKSPACE) ++n;                        // the merge
+  *launches = n;
+  return KDV_OK;
+}
+
 kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
   if (p == nullptr) return KDV_ERR_INVALID_ARG;
   const int impl = resolve_impl(p);
@@ -328,7 +344,7 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
     if (p->workspace == nullptr || p->workspace_bytes < need || !aligned16(p->workspace))
       return KDV_ERR_WORKSPACE;
   }
-  VerifyArgs a;
+  VerifyArgs a = {};
   a.q = p->q;
   a.q_row_stride = p->q_row_stride == 0 ? (int64_t)p->d_latent + p->d_rope : p->q_row_stride;
   a.kv = p->kv;

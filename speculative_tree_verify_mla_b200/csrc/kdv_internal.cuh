@@ -98,7 +98,9 @@ cudaError_t launch_combine_uniform(const float* o_part, const float* lse_part, i
                                    int64_t rows, int32_t d, float* o, float* lse,
                                    cudaStream_t stream);
 // Merges the workspace partials of a plan: fp32 o_k, or fp16 o_k when
-// p.part_f16 (then d must be 512).
+// p.part_f16 (then d must be 512). The fp16 merge is launched as a
+// programmatic dependent of the launch before it on `stream`, which must be
+// the tensor-core attention kernel that wrote the partials.
 cudaError_t launch_combine_plan(const void* ws_o, const float* ws_lse, const VerifyPlan& p,
                                 int32_t d, float* o, float* lse, cudaStream_t stream);
 

@@ -418,6 +418,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         for (int g = max(0, issued - KV_STAGES); g < issued; ++g)
           wait_bar(c, c.bar(B_KV_FULL + g % KV_STAGES), (g / KV_STAGES) & 1, true);
       }
+      // every load of this S CTA is issued: a programmatic dependent (the
+      // merge kernel) may launch as far as this CTA is concerned
+      asm volatile("griddepcontrol.launch_dependents;");
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------- pair MMA issuer: S[256 x 256] = Q[256 x 576] . K^T,
       // both operands in shared memory, into the two TMEM S buffers in turn:
@@ -744,6 +747,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       bad = named_bar_or(1, 2 * 128, bad);
       const bool have_o = n_ptiles > 0 && !bad;
       tc_fence_after();
+      // the merge kernel that follows (a programmatic dependent) may launch
+      // now; it waits for this grid to complete before it reads the partials
+      asm volatile("griddepcontrol.launch_dependents;");
       // ---------------- epilogue: o = O / l, lse = ln2 * (m + log2 l)
       const float l = *reinterpret_cast<volatile float*>(smem + OFF_STATS + r * 4);
       const float m = *reinterpret_cast<volatile float*>(smem + OFF_STATS + ROWS * 4 + r * 4);

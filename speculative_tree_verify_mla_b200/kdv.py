@@ -48,7 +48,7 @@ EXPORTED = ("kdv_status_string", "kdv_version", "kdv_tree_mask_build",
             "kdv_verify_attn_workspace", "kdv_verify_attn_plan", "kdv_verify_attn",
             "kdv_verify_attn_noalloc", "kdv_latent_f16", "kdv_combine", "kdv_tree_accept_workspace",
             "kdv_tree_accept", "kdv_absorb_q", "kdv_unabsorb_o", "kdv_tree_build",
-            "kdv_absorb_q_ex", "kdv_unabsorb_o_ex")
+            "kdv_absorb_q_ex", "kdv_unabsorb_o_ex", "kdv_verify_attn_launches")
 KDV_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
@@ -130,6 +130,8 @@ def load() -> ctypes.CDLL:
         lib.kdv_verify_attn_workspace.restype = c.c_int
         lib.kdv_verify_attn_plan.argtypes = [c.POINTER(VerifyParams), c.c_void_p, c.c_void_p]
         lib.kdv_verify_attn_plan.restype = c.c_int
+        lib.kdv_verify_attn_launches.argtypes = [c.POINTER(VerifyParams), c.POINTER(c.c_int32)]
+        lib.kdv_verify_attn_launches.restype = c.c_int
         lib.kdv_verify_attn.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
         lib.kdv_verify_attn.restype = c.c_int
         lib.kdv_verify_attn_noalloc.argtypes = [c.POINTER(VerifyParams), c.c_void_p]
@@ -231,6 +233,14 @@ def kdv_verify_attn_plan(params: VerifyParams):
     _check(load().kdv_verify_attn_plan(ctypes.byref(params), splits, ctypes.byref(items)),
            "kdv_verify_attn_plan")
     return [int(splits[i]) for i in range(params.batch)], int(items.value)
+
+
+def kdv_verify_attn_launches(params: VerifyParams) -> int:
+    """How many kernels kdv_verify_attn launches for these parameters."""
+    n = ctypes.c_int32(0)
+    _check(load().kdv_verify_attn_launches(ctypes.byref(params), ctypes.byref(n)),
+           "kdv_verify_attn_launches")
+    return int(n.value)
 
 
 def kdv_verify_attn(params: VerifyParams, stream=None) -> None:

@@ -38,7 +38,7 @@ def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4):
         assert kdv.status_string(s).startswith("KDV_")
     assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
-    assert kdv.kdv_version() == 121
+    assert kdv.kdv_version() == 122
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
@@ -133,6 +133,23 @@ def test_workspace_sizes(lib):
     assert kdv.kdv_verify_attn_workspace(p) == al(8 * 1024)
     # partials returned to the caller: no workspace
     assert kdv.kdv_verify_attn_workspace(_params(num_splits=3, return_partials=1)) == 0
+
+
+def test_launch_counts(lib):
+    """Kernels one kdv_verify_attn call launches (host planning only)."""
+    tc = dict(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC)
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=1)) == 1                  # SIMT, direct
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=3)) == 2                  # SIMT + merge
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=3, return_partials=1)) == 1
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=1, **tc)) == 2            # latent + TC
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=1, v16=0x10000, **tc)) == 1
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=3, v16=0x10000, **tc)) == 2
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=3, **tc)) == 3              # + merge
+    st = dict(tc, impl=kdv.KDV_IMPL_TC_STAGED, page_table=0x7000)
+    assert kdv.kdv_verify_attn_launches(_params(num_splits=1, v16=0x10000, **st)) == 2
+    n = ctypes.c_int32(0)
+    assert lib.kdv_verify_attn_launches(None, ctypes.byref(n)) == kdv.KDV_ERR_INVALID_ARG
+    assert lib.kdv_verify_attn_launches(ctypes.byref(_params()), None) == kdv.KDV_ERR_INVALID_ARG
 
 
 def test_mask_build_validation(lib):
