@@ -38,8 +38,12 @@ __global__ void __launch_bounds__(LF_THREADS)
 latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v16, uint8_t* __restrict__ staged,
                   int32_t* __restrict__ staged_off) {
   const int b = blockIdx.y;
-  // let a dependent attention grid launch now: it waits for this grid's
-  // completion before it reads the rows (griddepcontrol.wait)
+  // Launched as a programmatic dependent of whatever kernel precedes it on
+  // the stream (which may have written the pool or the page table): wait for
+  // it before any access. Then let the attention grid launch: it reads the
+  // fp16 rows only after this grid completes (griddepcontrol.wait), and
+  // everything else it reads was written before this point.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (staged_off != nullptr && blockIdx.x == 0 && b == 0)
     for (int i = threadIdx.x; i <= p.B; i += LF_THREADS)
@@ -117,10 +121,17 @@ cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v1
   int gx = (max_n + rows_per_cta - 1) / rows_per_cta;
   const int cap = (8 * 148 + p.B - 1) / p.B;
   if (gx > cap) gx = cap < 1 ? 1 : cap;
-  const dim3 grid((unsigned)gx, (unsigned)p.B);
-  latent_f16_kernel<<<grid, LF_THREADS, 0, stream>>>(a, p, static_cast<__half*>(v16), static_cast<uint8_t*>(staged),
-                                                      staged_off);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)p.B);
+  cfg.blockDim = dim3(LF_THREADS);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, latent_f16_kernel, a, p, static_cast<__half*>(v16), static_cast<uint8_t*>(staged),
+                            staged_off);
 }
 
 }  // namespace kdv
