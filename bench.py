@@ -298,6 +298,7 @@ class Problems:
         self.d_err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.trees = {}          # tree bytes -> (parent, tree_off, batch, max_T, mask)
         self.q, self.kv, self.o, self.lse, self.ws, self.params, self.tc_params = [], [], [], [], [], [], []
+        self.out = []
         self.page_table, self.kv_off, self.tree_off, self.keep = [], [], [], []
         self.splits, self.items = [], []
         self.v16, self.n_keys = [], []
@@ -313,8 +314,11 @@ class Problems:
             kv = torch.from_numpy(c.kv).to(torch.bfloat16).to(dev)
             pt = i32(c.page_table) if c.page_table is not None else None
             kv_off, tree_off, plen = i32(c.kv_off), i32(c.tree_off), i32(c.prefix_len)
-            o = torch.empty(c.rows, 512, dtype=torch.float32, device=dev)
-            lse = torch.empty(c.rows, dtype=torch.float32, device=dev)
+            # o and lse of a call in one allocation, so that a caller reading
+            # its results back to the host needs one copy, not two
+            out = torch.empty(c.rows * 513, dtype=torch.float32, device=dev)
+            o, lse = out[:c.rows * 512].view(c.rows, 512), out[c.rows * 512:]
+            self.out.append(out)
             common = dict(batch=c.batch, num_heads=c.H, d_latent=512, d_rope=64, scale=c.scale,
                           dtype=kdv.KDV_BF16, impl=impl_code, q=q, q_row_stride=576, kv=kv,
                           num_slots=kv.shape[0], page_table=pt, kv_off=kv_off, tree_off=tree_off,
@@ -655,16 +659,16 @@ def run_gpu(args):
                     slot = int(c.page_table[k0 + L + u])
                     rows_c.append((kv[slot:slot + 1], pin(kv[slot:slot + 1])))
         up_rows.append(rows_c)
-    h_o = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in prob.o]
-    h_l = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in prob.lse]
+    h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in prob.out]   # o then lse
     h2d = (sum(x.numel() * 4 for x in h_parent) + sum(x.numel() * 2 for x in h_q)
            + sum(h.numel() * 2 for rows_c in up_rows for _, h in rows_c))
-    d2h = sum(x.numel() * 4 for x in h_o) + sum(x.numel() * 4 for x in h_l)
+    d2h = sum(x.numel() * 4 for x in h_out)
 
     # The step pipelines its copies with the compute the way a serving loop
     # would: every call's inputs go up on a copy stream, each call starts once
-    # its own inputs have landed, and its o / lse come back on another copy
-    # stream while the next call runs. All copies stay inside the timed step.
+    # its own inputs have landed, and its o and lse (one allocation, so one
+    # copy) come back on another copy stream while the next call runs. All
+    # copies stay inside the timed step.
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_tree = torch.cuda.Event()
     ev_in = [torch.cuda.Event() for _ in prob.params]
@@ -690,8 +694,7 @@ def run_gpu(args):
             ev_out[l].record(stream)
             s_out.wait_event(ev_out[l])
             with torch.cuda.stream(s_out):
-                h_o[l].copy_(prob.o[l], non_blocking=True)
-                h_l[l].copy_(prob.lse[l], non_blocking=True)
+                h_out[l].copy_(prob.out[l], non_blocking=True)
         stream.wait_stream(s_out)
         stream.synchronize()
 
