@@ -67,6 +67,9 @@
 
 #include "kdv_internal.cuh"
 #include "sm100_ptx.cuh"
+#ifdef KDV_TRACE
+#include "kdv_trace.h"
+#endif
 
 namespace kdv {
 namespace {
@@ -153,6 +156,18 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+#ifdef KDV_TRACE
+// Tracing build (kdv_trace.h): CTA c writes the global timer at stage s
+// into kdv_trace_buf[c * KDV_TRACE_SLOTS + s].
+__device__ unsigned long long kdv_trace_buf[KDV_TRACE_CTAS * KDV_TRACE_SLOTS];
+__device__ __forceinline__ void trace_stamp(int slot) {
+  if (blockIdx.x < KDV_TRACE_CTAS) kdv_trace_buf[blockIdx.x * KDV_TRACE_SLOTS + slot] = globaltimer();
+}
+#define KDV_STAMP(slot) trace_stamp(slot)
+#else
+#define KDV_STAMP(slot) ((void)0)
+#endif
 
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;
@@ -335,6 +350,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+  if (threadIdx.x == 0) KDV_STAMP(KDV_TRACE_SETUP);
 
   if (s_side && leader && warp == 2 && lane == 0) {
     // device copies of the lengths against the host copies the plan used
@@ -450,6 +466,9 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         }
         if (!ok) break;
         tc_commit2_mc(c.bar(B_S_FULL + sb), S_PAIR);
+        if (i == 0) KDV_STAMP(KDV_TRACE_S_MMA_T0);
+        if (i == 1) KDV_STAMP(KDV_TRACE_S_MMA_T1);
+        if (i == n_stiles - 1) KDV_STAMP(KDV_TRACE_S_MMA_LAST);
       }
       tc_commit2_mc(c.bar(B_S_DRAIN), (uint16_t)(1u << rank));
       wait_bar(c, c.bar(B_S_DRAIN), 0, true);
@@ -478,6 +497,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       const uint32_t pbar0 = mapa(c.bar(B_P_FULL), o_rank);
       for (int i = 0; i < n_stiles; ++i) {
         ok = wait_warp(c, c.bar(B_S_FULL + (i & 1)), (i >> 1) & 1) && ok;
+        if (i == 0 && warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_SM0_T0_READY);
         const bool wok = __all_sync(0xffffffffu, ok);
         uint32_t sv[KEYS];
         if (wok) {
@@ -591,7 +611,10 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         l_part += lsum;
         // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
         if (ok) st_async_f32(pslot + P_BYTES + r * 4, hw == 0 ? alpha : 1.f, pbar);
+        if (i == 0 && warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_SM0_T0_DONE);
       }
+      if (warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_SM0_DONE);
+      if (warp == WG2_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_SM1_DONE);
       // final row statistics (sum of both halves) for the O side's epilogue
       volatile float* xs = xchg + 2 * ROWS;
       named_bar_sync(1, 2 * 128);
@@ -623,6 +646,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // grid was launched normally.
       asm volatile("griddepcontrol.wait;" ::: "memory");
       asm volatile("fence.proxy.async.global;" ::: "memory");
+      KDV_STAMP(KDV_TRACE_V_READY);
       for (int u = 0; u < n_sub; ++u) {
         const int st = u % V_STAGES;
         if (!wait_bar(c, c.bar(B_V_EMPTY + st), ((u / V_STAGES) & 1) ^ 1, true)) break;
@@ -667,6 +691,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         }
         if (!ok) break;
         tc_commit2_mc(c.bar(B_PV_DONE + slot), O_PAIR);
+        if (i == 0) KDV_STAMP(KDV_TRACE_PV_T0);
+        if (i == n_ptiles - 1) KDV_STAMP(KDV_TRACE_PV_LAST);
       }
       tc_commit2_mc(c.bar(B_O_DRAIN), (uint16_t)(1u << rank));
       wait_bar(c, c.bar(B_O_DRAIN), 0, true);
@@ -698,6 +724,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         for (int i = 0; i < n_ptiles; ++i) {
           const int slot = i % NP;
           const bool got = wait_warp(c, c.bar(B_P_FULL + slot), (i / NP) & 1);
+          if (i == 0 && warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_O_P0);
           if (!got && first_miss == n_ptiles) first_miss = i;
           ok = got && ok;
           fence_proxy_async_smem();      // P arrived by st.async; the pair's MMA reads it
@@ -750,6 +777,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
       // the merge kernel that follows (a programmatic dependent) may launch
       // now; it waits for this grid to complete before it reads the partials
       asm volatile("griddepcontrol.launch_dependents;");
+      if (warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_EPILOGUE);
       // ---------------- epilogue: o = O / l, lse = ln2 * (m + log2 l)
       const float l = *reinterpret_cast<volatile float*>(smem + OFF_STATS + r * 4);
       const float m = *reinterpret_cast<volatile float*>(smem + OFF_STATS + ROWS * 4 + r * 4);
@@ -823,6 +851,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           put_box(2 * ck + 1, col + 32, t1);
         }
       }
+      if (warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_STORED);
       if (warp_full && lane == 0) bulk_wait_group_read<0>();
       __syncwarp();
       if (eh == 0 && valid && a.lse != nullptr) a.lse[orow] = lse;
@@ -830,6 +859,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   }
 
   // ---- teardown ----------------------------------------------------------
+  if (warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_TEARDOWN);
   // After an abort (a wait that ran out) the O side stops waiting for P
   // tiles, so st.async bytes from the S pair could still be in flight toward
   // an O CTA when it reaches this point. So: a CTA whose abort flag is up
@@ -965,6 +995,29 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, verify_tc2_kernel<false>, tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
 }
+
+#ifdef KDV_TRACE
+}  // namespace kdv
+
+extern "C" {
+KDV_API kdv_status kdv_trace_clear(void* stream) {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, kdv::kdv_trace_buf) != cudaSuccess) return KDV_ERR_CUDA;
+  return cudaMemsetAsync(ptr, 0, sizeof(kdv::kdv_trace_buf), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDV_OK
+             : KDV_ERR_CUDA;
+}
+KDV_API kdv_status kdv_trace_read(uint64_t* host_dst, int64_t n_words) {
+  if (n_words < 0 || n_words > (int64_t)KDV_TRACE_CTAS * KDV_TRACE_SLOTS) return KDV_ERR_INVALID_ARG;
+  if (n_words == 0) return KDV_OK;
+  if (host_dst == nullptr) return KDV_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host_dst, kdv::kdv_trace_buf, (size_t)n_words * 8) == cudaSuccess ? KDV_OK
+                                                                                             : KDV_ERR_CUDA;
+}
+}  // extern "C"
+
+namespace kdv {
+#endif
 
 int tc2_max_active_clusters() {
   static int cached[64] = {};

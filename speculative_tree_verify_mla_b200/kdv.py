@@ -17,6 +17,16 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkdv.so")
+# the same library with the verify kernel's stage stamps (include/kdv_trace.h)
+TRACE_LIB_PATH = os.path.join(_PKG, "libkdv_trace.so")
+TRACE_EXPORTED = ("kdv_trace_clear", "kdv_trace_read")
+KDV_TRACE_CTAS = 1024
+KDV_TRACE_SLOTS = 16
+# stage slots, in kdv_trace.h order
+KDV_TRACE_STAGES = ("setup", "S mma t0 issued", "S mma t1 issued", "S mma last issued",
+                    "softmax0 sees S t0", "softmax0 pushed t0", "softmax0 done", "softmax1 done",
+                    "V rows ready", "PV t0 issued", "PV last issued", "O sees P t0",
+                    "epilogue start", "epilogue stored", "teardown")
 
 KDV_OK = 0
 KDV_ERR_INVALID_ARG = -1
@@ -158,8 +168,34 @@ def load() -> ctypes.CDLL:
         lib.kdv_unabsorb_o_ex.restype = c.c_int
         lib.kdv_tree_build.argtypes = [c.POINTER(BuildParams), c.c_void_p]
         lib.kdv_tree_build.restype = c.c_int
+        if hasattr(lib, "kdv_trace_read"):          # the tracing build
+            lib.kdv_trace_clear.argtypes = [c.c_void_p]
+            lib.kdv_trace_clear.restype = c.c_int
+            lib.kdv_trace_read.argtypes = [c.c_void_p, c.c_int64]
+            lib.kdv_trace_read.restype = c.c_int
         _lib = lib
     return _lib
+
+
+def use_trace_library() -> None:
+    """Make ``load()`` open libkdv_trace.so (call before the first load)."""
+    global LIB_PATH
+    if _lib is not None and LIB_PATH != TRACE_LIB_PATH:
+        raise RuntimeError("libkdv.so is already loaded in this process")
+    LIB_PATH = TRACE_LIB_PATH
+
+
+def kdv_trace_clear(stream=None) -> None:
+    _check(load().kdv_trace_clear(_stream(stream)), "kdv_trace_clear")
+
+
+def kdv_trace_read(n_ctas: int) -> np.ndarray:
+    """Stage stamps of the first n_ctas CTAs of the last traced launch:
+    uint64 [n_ctas][KDV_TRACE_SLOTS] global-timer ns (0 = stage not reached)."""
+    n_ctas = min(int(n_ctas), KDV_TRACE_CTAS)
+    out = np.zeros((n_ctas, KDV_TRACE_SLOTS), dtype=np.uint64)
+    _check(load().kdv_trace_read(out.ctypes.data, out.size), "kdv_trace_read")
+    return out
 
 
 def status_string(status: int) -> str:

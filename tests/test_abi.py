@@ -18,20 +18,42 @@ def lib():
     return kdv.load()
 
 
-def declared_symbols():
-    names = set()
-    for fn in os.listdir(os.path.join(ROOT, "include")):
-        if fn.endswith(".h"):
-            txt = open(os.path.join(ROOT, "include", fn)).read()
-            names |= set(re.findall(r"KDV_API[^;(]*?\b(kdv_\w+)\s*\(", txt))
-    return names
+def declared_symbols(header="kdv.h"):
+    txt = open(os.path.join(ROOT, "include", header)).read()
+    return set(re.findall(r"KDV_API[^;(]*?\b(kdv_\w+)\s*\(", txt))
 
 
 def test_exports_every_declared_symbol(lib):
+    assert sorted(fn for fn in os.listdir(os.path.join(ROOT, "include")) if fn.endswith(".h")) == \
+        ["kdv.h", "kdv_trace.h"]
     names = declared_symbols()
     assert names == set(kdv.EXPORTED), names
     for n in names:
         assert hasattr(lib, n), n
+    # the product library has none of the tracing build's entry points
+    for n in kdv.TRACE_EXPORTED:
+        assert not hasattr(lib, n), n
+
+
+def test_trace_build_exports_its_symbols():
+    """libkdv_trace.so exports everything kdv.h declares plus kdv_trace.h's."""
+    import ctypes as c
+    path = build.build_trace()
+    tlib = c.CDLL(path)
+    names = declared_symbols("kdv_trace.h")
+    assert names == set(kdv.TRACE_EXPORTED), names
+    for n in names | declared_symbols():
+        assert hasattr(tlib, n), n
+    txt = open(os.path.join(ROOT, "include", "kdv_trace.h")).read()
+    assert int(re.search(r"#define KDV_TRACE_CTAS (\d+)", txt).group(1)) == kdv.KDV_TRACE_CTAS
+    assert int(re.search(r"#define KDV_TRACE_SLOTS (\d+)", txt).group(1)) == kdv.KDV_TRACE_SLOTS
+    stages = re.findall(r"KDV_TRACE_\w+ = (\d+),?", txt)
+    assert [int(x) for x in stages] == list(range(len(kdv.KDV_TRACE_STAGES)))
+    # host-side argument checks need no GPU
+    assert tlib.kdv_trace_read(None, c.c_int64(-1)) == kdv.KDV_ERR_INVALID_ARG
+    assert tlib.kdv_trace_read(None, c.c_int64(kdv.KDV_TRACE_CTAS * kdv.KDV_TRACE_SLOTS + 1)) == \
+        kdv.KDV_ERR_INVALID_ARG
+    assert tlib.kdv_trace_read(None, c.c_int64(0)) == kdv.KDV_OK
 
 
 def test_status_strings(lib):
