@@ -218,7 +218,8 @@ KDV_API kdv_status kdv_verify_attn_launches(const kdv_verify_params* p, int32_t*
  * Absorbed Q.K^T over D_c + D_r dims, online softmax, P.V over the D_c latent
  * dims (V is the c_kv part of the same pool row), optional per-split LSE and
  * the split merge. Output o_lat is fp32 [sumT*H][D_c]; lse is the natural-log
- * log-sum-exp of the scaled logits. Requirements for the TC kernel: q, kv,
+ * log-sum-exp of the scaled logits. Requirements for the TC kernel: scale
+ * > 0 (KDV_ERR_UNSUPPORTED otherwise; AUTO then picks the SIMT kernel); q, kv,
  * o and o_part 16-byte aligned; q_row_stride*elem and (D_c+D_r)*elem
  * multiples of 16 bytes (KDV_ERR_INVALID_ARG otherwise).
  */

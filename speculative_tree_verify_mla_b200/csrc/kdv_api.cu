@@ -24,8 +24,10 @@ int device_sm_count() {
   return n;
 }
 
+// The tensor-core kernel: bf16, the Kimi / DeepSeek-V3 latent dims, and a
+// positive softmax scale (its row maxima are taken over unscaled logits).
 bool tc_shape_ok(const kdv_verify_params* p) {
-  return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64;
+  return p->dtype == KDV_BF16 && p->d_latent == 512 && p->d_rope == 64 && p->scale > 0.f;
 }
 
 bool is_tc(int impl) { return impl == KDV_IMPL_TC || impl == KDV_IMPL_TC_STAGED; }

@@ -516,13 +516,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         ok = ok && wok;
         const int key0 = stile_key(i) + hw * KEYS;
         float m_half = -INFINITY;
+        // the row max over raw logits, scaled once after: the scale is
+        // positive (checked on the host), so max(s) * sl2 = max(s * sl2),
+        // and the exp2 arguments below take the scale in one FMA
         if (valid && key0 + KEYS <= min(L, k_hi)) {
 #pragma unroll
-          for (int k = 0; k < KEYS; ++k) {
-            const float xk = __uint_as_float(sv[k]) * sl2;
-            sv[k] = __float_as_uint(xk);
-            m_half = fmaxf(m_half, xk);
-          }
+          for (int k = 0; k < KEYS; ++k) m_half = fmaxf(m_half, __uint_as_float(sv[k]));
         } else if (warp_rows) {
           // visibility of the tile's 128 keys as four 32-bit words: prefix
           // keys (j < L) inside the split, tree keys j = L+u with bit u of
@@ -544,11 +543,12 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
 #pragma unroll
           for (int k = 0; k < KEYS; ++k) {
             const bool vis = (vw[k >> 5] >> (k & 31)) & 1u;
-            const float xk = vis ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
+            const float xk = vis ? __uint_as_float(sv[k]) : -INFINITY;
             sv[k] = __float_as_uint(xk);
             m_half = fmaxf(m_half, xk);
           }
         }
+        m_half *= sl2;
         // Row max of the whole 256-key tile from both warpgroups -- needed
         // only if some row's reference max may move. One barrier vote
         // decides: when no half-tile max exceeds its row's m_run + TAU (and
@@ -591,8 +591,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             uint32_t w[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float p0 = ex2(__uint_as_float(sv[8 * ch + 2 * q]) - m_use);
-              const float p1 = ex2(__uint_as_float(sv[8 * ch + 2 * q + 1]) - m_use);
+              const float p0 = ex2(fmaf(__uint_as_float(sv[8 * ch + 2 * q]), sl2, -m_use));
+              const float p1 = ex2(fmaf(__uint_as_float(sv[8 * ch + 2 * q + 1]), sl2, -m_use));
               lsum += p0 + p1;
               w[q] = pack_f16x2(p0, p1);
             }

@@ -157,6 +157,19 @@ def test_workspace_sizes(lib):
     assert kdv.kdv_verify_attn_workspace(_params(num_splits=3, return_partials=1)) == 0
 
 
+def test_tensor_core_path_takes_positive_scales_only(lib):
+    """The TC kernel takes its row maxima over unscaled logits, so it needs
+    scale > 0: forced, a non-positive scale is refused; AUTO sends it to the
+    SIMT kernel (one launch, no fp16 latent pass)."""
+    tc = dict(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, num_splits=1)
+    for scale in (0.0, -0.1):
+        n = ctypes.c_size_t(0)
+        p = _params(impl=kdv.KDV_IMPL_TC, scale=scale, **tc)
+        assert lib.kdv_verify_attn_workspace(ctypes.byref(p), ctypes.byref(n)) == kdv.KDV_ERR_UNSUPPORTED
+        assert kdv.kdv_verify_attn_launches(_params(impl=kdv.KDV_IMPL_AUTO, scale=scale, **tc)) == 1
+    assert kdv.kdv_verify_attn_launches(_params(impl=kdv.KDV_IMPL_AUTO, scale=0.1, **tc)) == 2
+
+
 def test_launch_counts(lib):
     """Kernels one kdv_verify_attn call launches (host planning only)."""
     tc = dict(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC)
