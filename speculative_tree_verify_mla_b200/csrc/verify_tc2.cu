@@ -583,7 +583,10 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         // starts once warpgroup 0 has pushed its first 64 keys, so one
         // warpgroup's exp2 work overlaps the other's DSMEM pushes instead of
         // both computing, then both pushing.
-        float lsum = 0.f;
+        // row sum in two lanes (even and odd keys), added once at the end;
+        // the exp2 arguments two at a time (packed FMA)
+        float2 lsum2 = make_float2(0.f, 0.f);
+        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_use, -m_use);
         if (hw == 1) named_bar_sync(2, 2 * 128);
         if (warp_rows) {
 #pragma unroll
@@ -591,10 +594,11 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             uint32_t w[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float p0 = ex2(fmaf(__uint_as_float(sv[8 * ch + 2 * q]), sl2, -m_use));
-              const float p1 = ex2(fmaf(__uint_as_float(sv[8 * ch + 2 * q + 1]), sl2, -m_use));
-              lsum += p0 + p1;
-              w[q] = pack_f16x2(p0, p1);
+              const float2 x = fma_f32x2(make_float2(__uint_as_float(sv[8 * ch + 2 * q]),
+                                                     __uint_as_float(sv[8 * ch + 2 * q + 1])), sl2x2, negm);
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+              lsum2 = add_f32x2(lsum2, pp);
+              w[q] = pack_f16x2(pp.x, pp.y);
             }
             // no-swizzle K-major layout: keys 8ch..8ch+7 of row r at ch*2048 + r*16,
             // so a warp's 32 rows fill 512 contiguous bytes per store
@@ -608,7 +612,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
             for (int ch = 0; ch < KEYS / 8; ++ch) st_async_v4(pslot + ch * P_KCHUNK_BYTES + r * 16, 0u, 0u, 0u, 0u, pbar);
           }
         }
-        l_part += lsum;
+        l_part += lsum2.x + lsum2.y;
         // the O side rescales O before P tile 2i (slot 0); P tile 2i+1 needs none
         if (ok) st_async_f32(pslot + P_BYTES + r * 4, hw == 0 ? alpha : 1.f, pbar);
         if (i == 0 && warp == WG_FIRST_WARP && lane == 0) KDV_STAMP(KDV_TRACE_SM0_T0_DONE);
