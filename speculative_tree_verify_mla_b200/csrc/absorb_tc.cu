@@ -18,8 +18,10 @@
 //             staged by the threads in the same K-major swizzled layout.
 //   unabsorb: A = W_UV[h]^T, i.e. W_UV[h] read with v contiguous (MN-major):
 //             TMA boxes of [64 c][64 v]; B = the head's o_lat rows (fp32)
-//             split into bf16 hi = rn(o) and lo = rn(o - hi), two MMAs per
-//             K-step, so B carries ~16 significant bits and the product
+//             split into bf16 hi = rn(o) and lo = rn(o - hi), stacked as
+//             B rows [hi of the pass's nodes; lo of them], one MMA of twice
+//             the nodes per K-step and the two column halves added in the
+//             epilogue, so B carries ~16 significant bits and the product
 //             stays at fp32-accumulation accuracy (W_UV is exact in bf16).
 // The epilogue reads D with one TMEM lane per output row and one column per
 // node, so a warp's stores for one node cover 32 consecutive outputs.
@@ -73,14 +75,22 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, int dtype, flo
 }
 
 // Read D (this warp's 32 lanes, columns [0, n)) and write node t's value to
-// out[(t0 + t) * H + h][col0 + lane row].
+// out[(t0 + t) * H + h][col0 + lane row]; with lo_col > 0, node t's value is
+// the sum of columns t and lo_col + t.
 __device__ __forceinline__ void epilogue(uint32_t tmem, int n, bool ok, void* out, int64_t o_stride, int o_dtype,
-                                         int t0, int H, int h, int col0) {
+                                         int t0, int H, int h, int col0, int lo_col = 0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   for (int c0 = 0; c0 < n; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
+    if (lo_col > 0) {
+      uint32_t w[32];
+      tmem_ld32(tmem + lane_base + (uint32_t)(lo_col + c0), w);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
+    }
     tmem_wait_ld();
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
@@ -192,10 +202,9 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
   __shared__ uint32_t tmem_slot;
   const uint32_t base = align_1024(smem_u32(smem_raw));
   const int ncb = D_c / 64;
-  constexpr int BB = U_MAXN * 128;                 // one 64-c block of B (hi or lo)
+  constexpr int BB = 2 * U_MAXN * 128;             // one 64-c block of B: hi rows, then lo rows
   const uint32_t s_a = base;                       // ncb x ([64 c][64 v] x 2 v-blocks)
-  const uint32_t s_hi = base + ncb * BOX;          // ncb x [U_MAXN rows][64 c]
-  const uint32_t s_lo = s_hi + ncb * BB;
+  const uint32_t s_b = base + ncb * BOX;           // ncb x [2 npad rows][64 c]
   const int h = blockIdx.y, v0 = blockIdx.x * 128;
   const int warp = threadIdx.x >> 5;
   const uint32_t full = smem_u32(&bars[0]), done = smem_u32(&bars[1]);
@@ -209,7 +218,7 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
         tma_load_2d(s_a + cb * BOX + vb * (BOX / 2), &tmap_w, full, v0 + vb * 64, h * D_c + cb * 64);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_slot), tmem_cols_for(U_MAXN));
+    tmem_alloc(smem_u32(&tmem_slot), tmem_cols_for(2 * U_MAXN));
     tmem_relinquish();
   }
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -254,9 +263,9 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
           hi[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
           lo[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
         }
-        const uint32_t off = cb * BB + t * 128 + ((ch ^ (t & 7)) << 4);
-        st_shared_v4(s_hi + off, hi[0], hi[1], hi[2], hi[3]);
-        st_shared_v4(s_lo + off, lo[0], lo[1], lo[2], lo[3]);
+        const int tl = npad + t;                    // the lo row of node t
+        st_shared_v4(s_b + cb * BB + t * 128 + ((ch ^ (t & 7)) << 4), hi[0], hi[1], hi[2], hi[3]);
+        st_shared_v4(s_b + cb * BB + tl * 128 + ((ch ^ (tl & 7)) << 4), lo[0], lo[1], lo[2], lo[3]);
       }
     }
     fence_proxy_async_smem();
@@ -267,13 +276,12 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
       if (ok) {
         // A MN-major: 64-v blocks BOX/2 apart, 8-row (c) groups 1024 B apart,
         // 16 c per K-step = 2048 B
-        const uint32_t idesc = idesc_bf16_f32(128, npad, true, false);
+        const uint32_t idesc = idesc_bf16_f32(128, 2 * npad, true, false);
         for (int cb = 0; cb < ncb; ++cb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t adesc = sw128_desc(s_a + cb * BOX + kk * 2048, BOX / 2, 1024);
-            mma_ss(tmem, adesc, sw128_desc(s_hi + cb * BB + kk * 32, 16, 1024), idesc, (cb > 0 || kk > 0) ? 1u : 0u);
-            mma_ss(tmem, adesc, sw128_desc(s_lo + cb * BB + kk * 32, 16, 1024), idesc, 1u);
+            mma_ss(tmem, adesc, sw128_desc(s_b + cb * BB + kk * 32, 16, 1024), idesc, (cb > 0 || kk > 0) ? 1u : 0u);
           }
       }
       tc_commit(done);
@@ -281,14 +289,14 @@ unabsorb_o_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, int32_t rows_pe
     const bool landed = tc_wait(done, pass & 1);
     ok = __syncthreads_and(ok && landed) != 0;
     tc_fence_after();
-    epilogue(tmem, n, ok, out, o_stride, o_dtype, t0, H, h, v0);
+    epilogue(tmem, n, ok, out, o_stride, o_dtype, t0, H, h, v0, npad);
     tc_fence_before();
     __syncthreads();
   }
   if (threadIdx.x == 0 && rows_per_head > 0 && !ok) tc_wait(full, 0);
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols_for(U_MAXN));
+    tmem_dealloc(tmem, tmem_cols_for(2 * U_MAXN));
   }
 }
 
