@@ -94,12 +94,18 @@ typedef enum {
 #define KDV_IMPL_SIMT 1
 #define KDV_IMPL_TC 2
 #define KDV_IMPL_TC_1SM 3
-/* TC_STAGED: the 2-SM kernel over a paged pool, first copying every request's
- * rows (in logical order) into a contiguous region of the workspace -- in the
- * same pass that writes the fp16 rows -- and then reading them with tiled
- * TMA boxes instead of four-row gathers. Faster for paged pools at the price
- * of workspace = (sum of L_b + T_b) x (D_c + D_r) x 2 bytes more; AUTO's
- * choice for paged pools. Without a page table it is KDV_IMPL_TC. */
+/* TC_STAGED: the 2-SM kernel over a paged pool that reads every key with
+ * tiled TMA boxes instead of four-row gathers: the pass that writes the fp16
+ * rows (in logical order) also copies each key's k_rope into a contiguous
+ * region of the workspace and writes q_lat in fp16, and Q.K^T then runs over
+ * the latent dims in fp16 and over the rope dims in bf16. bf16 -> fp16 is
+ * exact for 2^-14 <= |x| < 65536; smaller magnitudes round to fp16
+ * subnormals (so results can differ from KDV_IMPL_TC by a few fp32 ulps), and
+ * a q_lat value beyond that range sets KDV_DERR_RANGE, as a c_kv value does.
+ * Faster for paged pools at the price of workspace = (sum of L_b + T_b) x
+ * D_r x 2 + (sum of T_b) x H x D_c x 2 bytes more (plus the batch's
+ * offsets, each region rounded up to 256 B); AUTO's choice for paged pools.
+ * Without a page table it is KDV_IMPL_TC. */
 #define KDV_IMPL_TC_STAGED 4
 
 #define KDV_MAX_TREE 64    /* nodes per tree (one 64-bit mask word)          */
@@ -113,7 +119,9 @@ KDV_API const char* kdv_status_string(kdv_status s);
  * the 100 set (mask build, verify, no-alloc verify, combine); 120 adds
  * kdv_latent_f16, the wait_limit_ns and v16 fields of kdv_verify_params,
  * KDV_DERR_RANGE, and retires KDV_IMPL_TC_1SM; 121 adds kdv_absorb_q_ex /
- * kdv_unabsorb_o_ex; 122 adds kdv_verify_attn_launches. */
+ * kdv_unabsorb_o_ex; 122 adds kdv_verify_attn_launches; 123: KDV_IMPL_TC_STAGED
+ * stages k_rope and q_lat in fp16 instead of whole bf16 rows (another
+ * workspace size). */
 KDV_API int32_t kdv_version(void);
 
 /*

@@ -252,10 +252,11 @@ kdv_status make_plan(const kdv_verify_params* p, int impl, VerifyPlan* plan, siz
   }
   if (is_tc2(impl) && p->v16 == nullptr) *ws_bytes = v16_offset(*plan, p->d_latent) + align256(v16_bytes(*plan));
   if (staged_paged(p, impl)) {
-    // after the fp16 rows: staged row offsets [B+1], then the staged rows
+    // after the fp16 rows: staged row offsets [B+1], the staged k_rope rows
+    // [keys][D_r], then q_lat in fp16 [total_rows][D_c]
     const size_t n_keys = (size_t)plan_keys(*plan);
     *ws_bytes = align256(*ws_bytes) + align256((size_t)(B + 1) * sizeof(int32_t)) +
-                n_keys * (size_t)(p->d_latent + p->d_rope) * 2;
+                align256(n_keys * (size_t)p->d_rope * 2) + (size_t)plan->total_rows * p->d_latent * 2;
   }
   return KDV_OK;
 }
@@ -277,7 +278,7 @@ const char* kdv_status_string(kdv_status s) {
   return "KDV_ERR_UNKNOWN";
 }
 
-int32_t kdv_version(void) { return 122; }
+int32_t kdv_version(void) { return 123; }
 
 kdv_status kdv_tree_mask_build(const int32_t* parent, const int32_t* tree_off, int32_t batch,
                                int32_t max_T, uint64_t* mask, int32_t* depth, int32_t* d_err,
@@ -383,6 +384,7 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
   void* own_v16 = nullptr;
   void* staged = nullptr;
   int32_t* staged_off = nullptr;
+  void* q16 = nullptr;
   if (is_tc2(impl) && v16 == nullptr) {
     own_v16 = static_cast<char*>(p->workspace) + v16_offset(plan, p->d_latent);
     v16 = own_v16;
@@ -392,15 +394,19 @@ kdv_status kdv_verify_attn(const kdv_verify_params* p, void* stream) {
                    (p->v16 == nullptr ? align256(v16_bytes(plan)) : 0);
     staged_off = reinterpret_cast<int32_t*>(region);
     staged = region + align256((size_t)(plan.B + 1) * sizeof(int32_t));
+    q16 = static_cast<char*>(staged) + align256((size_t)plan_keys(plan) * p->d_rope * 2);
   }
   if (own_v16 != nullptr || staged != nullptr) {
-    if (launch_latent_f16(a, plan, own_v16, staged, staged_off, s) != cudaSuccess) return KDV_ERR_CUDA;
+    if (launch_latent_f16(a, plan, own_v16, staged, staged_off, q16, s) != cudaSuccess) return KDV_ERR_CUDA;
   }
   if (staged != nullptr) {
+    // the keys in logical order: latent dims from the fp16 rows, k_rope
+    // from the staged rows, queries' latent dims from q16
     a.kv = staged;
     a.num_slots = plan_keys(plan);
     a.page_table = nullptr;
     a.kv_off = staged_off;
+    a.q16 = q16;
   }
   // The attention kernel may start while the latent pass still runs when
   // that pass writes only the fp16 rows (not a staged pool the S side reads).
@@ -433,7 +439,7 @@ kdv_status kdv_latent_f16(const kdv_verify_params* p, void* v16, void* stream) {
   a.D_c = q.d_latent;
   a.D_r = q.d_rope;
   a.d_err = q.d_err;
-  return cuda_status(launch_latent_f16(a, plan, v16, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_latent_f16(a, plan, v16, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
 kdv_status kdv_combine(const float* o_part, const float* lse_part, int32_t S, int64_t rows,

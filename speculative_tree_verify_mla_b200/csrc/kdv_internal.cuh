@@ -53,6 +53,11 @@ struct VerifyArgs {
   float* lse;        // matching lse array (may be null in OUT_DIRECT)
   int32_t* d_err;
   uint64_t wait_limit_ns;   // pipeline-wait bound of the TC kernel (0 = its default, 1 s)
+  // Staged paged pool (TC kernel): q_lat as fp16 [total_rows][512], written
+  // by the latent pass. When set, the S pair reads Q.K^T's latent dims in
+  // fp16 -- the queries from here, the keys from the fp16 latent rows -- and
+  // only k_rope from kv, which then holds [keys][D_r] bf16 rows.
+  void* q16;
 };
 
 // Where the (request b, split s, local row r) result goes, in rows of D_c.
@@ -87,10 +92,12 @@ cudaError_t launch_verify_simt(const VerifyArgs& a, const VerifyPlan& p, int32_t
 // dependent and only the V loads wait for it (griddepcontrol.wait).
 cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const void* v16, int64_t v16_rows,
                               bool after_latent, cudaStream_t stream);
-// Writes the fp16 latent rows (v16, nullable) and, for a paged pool, the
-// staged bf16 rows with their offsets (staged / staged_off, nullable).
+// Writes the fp16 latent rows (v16, nullable) and, for a staged paged pool,
+// the k_rope rows [keys][D_r] with their offsets (staged / staged_off) and
+// q_lat as fp16 [total_rows][512] (q16): those three are all given or all
+// null (else cudaErrorInvalidValue).
 cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v16, void* staged, int32_t* staged_off,
-                              cudaStream_t stream);
+                              void* q16, cudaStream_t stream);
 // Work items (4-CTA clusters) of the TC kernel that fit on the device at
 // once, i.e. one wave; 0 when the query fails (no device).
 int tc2_max_active_clusters();

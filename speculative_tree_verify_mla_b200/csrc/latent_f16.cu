@@ -14,15 +14,19 @@
 // exact for 2^-14 <= |x| < 65536; smaller values round to fp16 subnormals;
 // |x| >= 65536 (or inf / NaN) is reported as KDV_DERR_RANGE.
 //
-// A paged pool can also be staged in the same pass: with `staged` given, the
-// whole bf16 row (c_kv || k_rope, 1152 bytes) is copied to staged row
-// v16_base[b] + j as well, and staged_off[b] = v16_base[b], so the verify
-// kernel reads the request's keys with tiled TMA boxes instead of gathers.
+// A paged pool can also be staged in the same pass: with `staged` given,
+// the row's k_rope (D_r = 64 bf16, 128 bytes) is copied to staged row
+// v16_base[b] + j, staged_off[b] = v16_base[b], and q_lat is written as fp16
+// to q16 [total_rows][512]. The verify kernel then reads the request's keys
+// with tiled TMA boxes instead of gathers: their latent dims from the fp16
+// rows (Q.K^T over them in fp16: the same products as bf16 except where an
+// input below 2^-14 in magnitude was rounded to an fp16 subnormal), their
+// rope dims from the staged rows.
 //
-// HBM-bound: 1 KB read and 1 KB written per key (+1152 B written when
-// staging). One warp per key row, lane l owning dims [16 l, 16 l + 16) (and,
-// for lanes 0-7, k_rope bytes [16 l, 16 l + 16)); each warp keeps four rows'
-// loads in flight.
+// HBM-bound: 1 KB read and 1 KB written per key (+128 B read and written
+// when staging). One warp per key row, lane l owning dims [16 l, 16 l + 16)
+// (and, for lanes 0-7, k_rope bytes [16 l, 16 l + 16)); each warp keeps four
+// rows' loads in flight.
 #include <cuda_fp16.h>
 
 #include "kdv_internal.cuh"
@@ -34,9 +38,12 @@ namespace {
 constexpr int LF_THREADS = 256;
 constexpr int LF_ROWS = 4;           // rows in flight per warp
 
+// STAGED: staged, staged_off and q16 are given (a paged pool staged in this
+// pass); otherwise all three are null and their code is compiled out
+template <bool STAGED>
 __global__ void __launch_bounds__(LF_THREADS)
 latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v16, uint8_t* __restrict__ staged,
-                  int32_t* __restrict__ staged_off) {
+                  int32_t* __restrict__ staged_off, __half* __restrict__ q16) {
   const int b = blockIdx.y;
   // Launched as a programmatic dependent of whatever kernel precedes it on
   // the stream (which may have written the pool or the page table): wait for
@@ -45,7 +52,7 @@ latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v
   // everything else it reads was written before this point.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (staged_off != nullptr && blockIdx.x == 0 && b == 0)
+  if (STAGED && blockIdx.x == 0 && b == 0)
     for (int i = threadIdx.x; i <= p.B; i += LF_THREADS)
       staged_off[i] = i < p.B ? p.v16_base[i] : p.v16_base[p.B - 1] + p.L[p.B - 1] + p.T[p.B - 1];
   const int n = p.L[b] + p.T[b];
@@ -70,7 +77,7 @@ latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v
         const uint4* src = reinterpret_cast<const uint4*>(kv + row * (int64_t)((a.D_c + a.D_r) * 2) + lane * 32);
         x[r][0] = ptx::ldg_nc_v4(src);
         x[r][1] = ptx::ldg_nc_v4(src + 1);
-        if (staged != nullptr && lane < 8)
+        if (STAGED && lane < 8)
           xr[r] = ptx::ldg_nc_v4(reinterpret_cast<const uint4*>(kv + row * (int64_t)((a.D_c + a.D_r) * 2) + 1024 +
                                                                    lane * 16));
       }
@@ -94,12 +101,26 @@ latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v
           dst[0] = y[0];
           dst[1] = y[1];
         }
-        if (staged != nullptr) {
-          uint4* srow = reinterpret_cast<uint4*>(staged + out_row * (int64_t)((a.D_c + a.D_r) * 2));
-          srow[2 * lane] = x[r][0];
-          srow[2 * lane + 1] = x[r][1];
-          if (lane < 8) srow[64 + lane] = xr[r];
-        }
+        if (STAGED && lane < 8)
+          reinterpret_cast<uint4*>(staged + out_row * (int64_t)(a.D_r * 2))[lane] = xr[r];
+      }
+    }
+  }
+  if (STAGED) {
+    // q_lat as fp16: one warp per query row, over all CTAs of the grid
+    const int64_t wid = ((int64_t)b * gridDim.x + blockIdx.x) * (LF_THREADS / 32) + warp;
+    const int64_t nw = (int64_t)gridDim.x * gridDim.y * (LF_THREADS / 32);
+    for (int64_t row = wid; row < p.total_rows; row += nw) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(a.q) + row * a.q_row_stride * 2 +
+                                                        lane * 32);
+      uint4 w[2] = {ptx::ldg_nc_v4(src), ptx::ldg_nc_v4(src + 1)};
+      uint4* dst = reinterpret_cast<uint4*>(q16 + row * 512 + lane * 16);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        range |= ptx::bf16x2_beyond_f16(w[h].x) | ptx::bf16x2_beyond_f16(w[h].y) | ptx::bf16x2_beyond_f16(w[h].z) |
+                 ptx::bf16x2_beyond_f16(w[h].w);
+        dst[h] = make_uint4(ptx::bf16x2_to_f16x2(w[h].x), ptx::bf16x2_to_f16x2(w[h].y), ptx::bf16x2_to_f16x2(w[h].z),
+                            ptx::bf16x2_to_f16x2(w[h].w));
       }
     }
   }
@@ -111,15 +132,19 @@ latent_f16_kernel(const VerifyArgs a, const VerifyPlan p, __half* __restrict__ v
 }  // namespace
 
 cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v16, void* staged, int32_t* staged_off,
-                              cudaStream_t stream) {
-  if (a.D_c != 512 || (staged != nullptr && a.D_r != 64)) return cudaErrorInvalidValue;
+                              void* q16, cudaStream_t stream) {
+  const bool stage = staged != nullptr;
+  if (a.D_c != 512 || (stage && a.D_r != 64) || (staged_off != nullptr) != stage || (q16 != nullptr) != stage)
+    return cudaErrorInvalidValue;
   int max_n = 0;
   for (int b = 0; b < p.B; ++b) max_n = max_n > p.L[b] + p.T[b] ? max_n : p.L[b] + p.T[b];
   if (max_n == 0) return cudaSuccess;
   const int rows_per_cta = (LF_THREADS / 32) * LF_ROWS;
-  // enough CTAs in flight to keep HBM busy, fewer for a short request
+  // enough CTAs in flight to keep HBM busy, fewer for a short request; at
+  // 200k keys a cap of 16 CTAs per SM streams ~10% faster than 8 (more
+  // waves of short-lived CTAs even out the rows per CTA)
   int gx = (max_n + rows_per_cta - 1) / rows_per_cta;
-  const int cap = (8 * 148 + p.B - 1) / p.B;
+  const int cap = (16 * 148 + p.B - 1) / p.B;
   if (gx > cap) gx = cap < 1 ? 1 : cap;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)gx, (unsigned)p.B);
@@ -130,8 +155,8 @@ cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v1
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, latent_f16_kernel, a, p, static_cast<__half*>(v16), static_cast<uint8_t*>(staged),
-                            staged_off);
+  return cudaLaunchKernelEx(&cfg, stage ? latent_f16_kernel<true> : latent_f16_kernel<false>, a, p, static_cast<__half*>(v16), static_cast<uint8_t*>(staged),
+                            staged_off, static_cast<__half*>(q16));
 }
 
 }  // namespace kdv

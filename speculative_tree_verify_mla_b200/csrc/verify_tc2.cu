@@ -145,6 +145,7 @@ static_assert(B_O_DRAIN < NUM_BARS, "barrier slots");
 
 constexpr uint16_t S_PAIR = 0x3, O_PAIR = 0xC;     // cluster CTA masks
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(256, 256, false, false);
+constexpr uint32_t IDESC_QK16 = idesc_f16_f32(256, 256, false, false);   // latent dims in fp16 (staged pool)
 constexpr uint32_t IDESC_PV = idesc_f16_f32(256, 256, false, true);   // fp16 P and V
 
 constexpr int THREADS = 384;
@@ -267,10 +268,13 @@ __device__ __forceinline__ int32_t paged_slot(const VerifyArgs& a, int64_t kv_ba
   return s;
 }
 
-template <bool PAGED>
+// PAGED: the keys gathered through the page table (bf16); LAT16: a staged
+// pool, Q.K^T's latent dims read in fp16 (never both)
+template <bool PAGED, bool LAT16>
 __global__ void __launch_bounds__(THREADS, 1) __cluster_dims__(4, 1, 1)
 verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_v,
                   const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_o,
+                  const __grid_constant__ CUtensorMap tmap_l16, const __grid_constant__ CUtensorMap tmap_q16,
                   const int o_tma, const VerifyArgs a, const VerifyPlan p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -304,6 +308,7 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
   auto stile_key = [&](int i) { return k_lo + i * STILE; };
   const int n_ptiles = 2 * n_stiles;
   const int64_t kv_base = a.kv_off[b];
+  constexpr bool lat16 = LAT16 && !PAGED;
 
   // ---- setup -------------------------------------------------------------
   if (threadIdx.x == 0) {
@@ -389,7 +394,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
         if (lane == 0)
           for (; q_issued < upto; ++q_issued) {
             if (leader) mbar_arrive_expect_tx(c.bar(B_Q_FULL + q_issued), 2 * QBLOCK_BYTES);
-            tma_load_2d_pair(base + OFF_Q + q_issued * QBLOCK_BYTES, &tmap_q,
+            tma_load_2d_pair(base + OFF_Q + q_issued * QBLOCK_BYTES,
+                             lat16 && q_issued < QK_BLOCKS - 1 ? &tmap_q16 : &tmap_q,
                              mapa(c.bar(B_Q_FULL + q_issued), lead_rank), q_issued * 64, qy);
           }
       };
@@ -421,9 +427,13 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           tma_gather4_pair(dst + lane * 512, &tmap_kv, fb, blk * 64, slot[0], slot[1], slot[2], slot[3]);
         } else {
           const int32_t y = (int32_t)(kv_base + stile_key(tile) + (int)half * HKEYS);
+          // staged pool: latent K-blocks from the fp16 rows, the rope block
+          // from the staged k_rope rows (its columns start at 0 there)
+          auto kv_map = [&](int e) { return lat16 && e < QK_BLOCKS - 1 ? &tmap_l16 : &tmap_kv; };
+          auto kv_x = [&](int e) { return lat16 && e == QK_BLOCKS - 1 ? 0 : e * 64; };
           if (blk == 0 && tile + 1 < n_stiles)
-            for (int e = 0; e < QK_BLOCKS; ++e) tma_prefetch_l2(&tmap_kv, e * 64, y + STILE);
-          tma_load_2d_pair(dst, &tmap_kv, fb, blk * 64, y);
+            for (int e = 0; e < QK_BLOCKS; ++e) tma_prefetch_l2(kv_map(e), kv_x(e), y + STILE);
+          tma_load_2d_pair(dst, kv_map(blk), fb, kv_x(blk), y);
         }
         issued = g + 1;
         if (g == KV_STAGES - 1) issue_q(QK_BLOCKS);
@@ -460,8 +470,8 @@ verify_tc2_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_cons
           const uint32_t kb = base + OFF_KV + st * KBLOCK_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma2_ss(d, sw128_desc(qb + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024), IDESC_QK,
-                    (blk > 0 || kk > 0) ? 1u : 0u);
+            mma2_ss(d, sw128_desc(qb + kk * 32, 16, 1024), sw128_desc(kb + kk * 32, 16, 1024),
+                    lat16 && blk < QK_BLOCKS - 1 ? IDESC_QK16 : IDESC_QK, (blk > 0 || kk > 0) ? 1u : 0u);
           tc_commit2_mc(c.bar(B_KV_EMPTY + st), S_PAIR);
         }
         if (!ok) break;
@@ -925,16 +935,18 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
   if (enc == nullptr) return cudaErrorNotSupported;
   if (a.num_slots < 1 || a.num_slots > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
   if (p.total_rows < 1) return cudaErrorInvalidValue;
-  auto make = [&](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t pitch_elems, uint32_t box_rows) {
-    const cuuint64_t dims[2] = {(cuuint64_t)DQ, (cuuint64_t)rows};
+  // 16-bit [rows][cols] with a row pitch, in 64-column boxes of box_rows rows
+  auto make = [&](CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t pitch_elems, uint32_t box_rows,
+                  uint64_t cols = DQ, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)pitch_elems * 2};
     const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+    return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   };
-  CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o;
+  CUtensorMap tmap_kv, tmap_v, tmap_q, tmap_o, tmap_l16, tmap_q16;
   const bool paged = a.page_table != nullptr;
   if (v16 == nullptr || v16_rows < 1 || v16_rows > (int64_t)0x7fffffff) return cudaErrorInvalidValue;
   // V: the fp16 latent rows [v16_rows][512] in 32-row boxes
@@ -948,9 +960,22 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : HKEYS) != CUDA_SUCCESS ||
-      make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
+  if (make(&tmap_q, a.q, (uint64_t)p.total_rows, (uint64_t)a.q_row_stride, ROWS) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (a.q16 != nullptr) {
+    // staged pool: kv holds only k_rope [keys][D_r]; the keys' latent dims
+    // come from the fp16 rows, the queries' from q16, both in 128-row boxes
+    if (paged || a.D_r != 64 ||
+        make(&tmap_kv, a.kv, (uint64_t)a.num_slots, (uint64_t)a.D_r, HKEYS, (uint64_t)a.D_r) != CUDA_SUCCESS ||
+        make(&tmap_l16, v16, (uint64_t)v16_rows, DC, HKEYS, DC, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS ||
+        make(&tmap_q16, a.q16, (uint64_t)p.total_rows, DC, ROWS, DC, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    if (make(&tmap_kv, a.kv, (uint64_t)a.num_slots, DQ, paged ? 1 : HKEYS) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    tmap_l16 = tmap_kv;     // unused
+    tmap_q16 = tmap_q;
+  }
   // output rows for the epilogue's TMA stores
   int64_t out_rows = 0;
   for (int b = 0; b < p.B; ++b)
@@ -972,19 +997,18 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  using KernelFn = decltype(&verify_tc2_kernel<false, false>);
+  const KernelFn kernels[3] = {verify_tc2_kernel<false, false>, verify_tc2_kernel<true, false>,
+                               verify_tc2_kernel<false, true>};
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(verify_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(verify_tc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    for (int i = 0; e == cudaSuccess && i < 3; ++i)
+      e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  if (paged) {
-    verify_tc2_kernel<true><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
-    return cudaGetLastError();
-  }
-  if (!after_latent) {
-    verify_tc2_kernel<false><<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
+  const KernelFn kern = kernels[paged ? 1 : a.q16 != nullptr ? 2 : 0];
+  if (paged || !after_latent) {
+    kern<<<4 * p.n_items, THREADS, SMEM_BYTES, stream>>>(tmap_kv, tmap_v, tmap_q, tmap_o, tmap_l16, tmap_q16, o_tma, a, p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -997,7 +1021,7 @@ cudaError_t launch_verify_tc2(const VerifyArgs& a, const VerifyPlan& p, const vo
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, verify_tc2_kernel<false>, tmap_kv, tmap_v, tmap_q, tmap_o, o_tma, a, p);
+  return cudaLaunchKernelEx(&cfg, kern, tmap_kv, tmap_v, tmap_q, tmap_o, tmap_l16, tmap_q16, o_tma, a, p);
 }
 
 #ifdef KDV_TRACE
@@ -1028,7 +1052,7 @@ int tc2_max_active_clusters() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 0; }
   if (cached[dev] > 0) return cached[dev];
-  if (cudaFuncSetAttribute(verify_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+  if (cudaFuncSetAttribute(verify_tc2_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -1044,7 +1068,7 @@ int tc2_max_active_clusters() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, verify_tc2_kernel<false>, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
+  if (cudaOccupancyMaxActiveClusters(&n, verify_tc2_kernel<false, false>, &cfg) != cudaSuccess) { cudaGetLastError(); return 0; }
   cached[dev] = n;
   return n;
 }

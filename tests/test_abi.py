@@ -60,7 +60,7 @@ def test_status_strings(lib):
     for s in (0, -1, -2, -3, -4):
         assert kdv.status_string(s).startswith("KDV_")
     assert kdv.status_string(-99) == "KDV_ERR_UNKNOWN"
-    assert kdv.kdv_version() == 122
+    assert kdv.kdv_version() == 123
 
 
 @pytest.mark.parametrize("cls,cname", [(kdv.VerifyParams, "kdv_verify_params"),
@@ -310,10 +310,11 @@ def test_tree_build_validation(lib):
 def test_staged_workspace_size(lib):
     al = lambda x: ((x + 255) // 256) * 256
     # forced single split (no merge region): the fp16 latent rows, then the
-    # staged offsets [B+1], then the staged rows
+    # staged offsets [B+1], the staged k_rope rows, then q_lat in fp16
+    # (T * H = 3 * 4 rows)
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC_STAGED,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
-    assert kdv.kdv_verify_attn_workspace(p) == al(103 * 1024) + 256 + 103 * 576 * 2
+    assert kdv.kdv_verify_attn_workspace(p) == al(103 * 1024) + 256 + al(103 * 64 * 2) + 3 * 4 * 512 * 2
     # reading the pool through the page table needs only the fp16 rows
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])

@@ -151,17 +151,21 @@ def test_tc_auto_stages_a_paged_pool():
 # ---------------------------------------------------------------------------
 # Paged KV through a staged contiguous copy (KDV_IMPL_TC_STAGED).
 
-def test_tc_staged_equals_gather_bit_for_bit():
-    """Staging the rows in logical order and reading them with tiled boxes
-    gives exactly what the four-row gathers give."""
+def test_tc_staged_equals_gather():
+    """Staging in logical order and reading with tiled boxes gives what the
+    four-row gathers give, up to the staged path's fp16 Q.K^T over the
+    latent dims: exact except for inputs below 2^-14 in magnitude, which fp16
+    holds as subnormals (a few fp32 ulps on a small fraction of outputs)."""
     parents = [datagen.random_tree(T, np.random.default_rng(T + 7)) for T in (13, 16, 9)]
     case = datagen.make_case("st", **datagen.KIMI, prefix_len=[2100, 333, 4097], parents=parents,
                              seed=41, paged=True)
     for splits in (0, 1, 3):
         og, lg = _run(case, kdv.KDV_IMPL_TC, splits=splits)
         os_, ls_ = _run(case, kdv.KDV_IMPL_TC_STAGED, splits=splits)
-        np.testing.assert_array_equal(og, os_)
-        np.testing.assert_array_equal(lg, ls_)
+        diff = np.abs(og - os_)
+        assert np.count_nonzero(diff) <= 2e-3 * diff.size
+        assert diff.max() <= 1e-4 * float(np.sqrt(np.mean(og.astype(np.float64) ** 2)))
+        assert np.abs(lg - ls_).max() <= 1e-5
     o_ref, lse_ref = oracle.verify_case(case)
     assert_parity(os_, ls_, o_ref, lse_ref)
 
