@@ -141,8 +141,9 @@ cudaError_t launch_latent_f16(const VerifyArgs& a, const VerifyPlan& p, void* v1
   if (max_n == 0) return cudaSuccess;
   const int rows_per_cta = (LF_THREADS / 32) * LF_ROWS;
   // enough CTAs in flight to keep HBM busy, fewer for a short request; at
-  // 200k keys a cap of 16 CTAs per SM streams ~10% faster than 8 (more
-  // waves of short-lived CTAs even out the rows per CTA)
+  // 200k keys a grid capped at 16 x 148 CTAs streams ~10% faster than one
+  // capped at 8 x 148 (more waves of short-lived CTAs even out the rows per
+  // CTA)
   int gx = (max_n + rows_per_cta - 1) / rows_per_cta;
   const int cap = (16 * 148 + p.B - 1) / p.B;
   if (gx > cap) gx = cap < 1 ? 1 : cap;
