@@ -45,13 +45,16 @@ def test_latent_f16_rows_equal_the_cast(paged):
     assert torch.equal(v16.view(torch.int16), want.view(torch.int16))
 
 
+@pytest.mark.parametrize("impl", [kdv.KDV_IMPL_TC, kdv.KDV_IMPL_TC_STAGED])
 @pytest.mark.parametrize("splits", [0, 1])
-def test_caller_rows_give_the_same_bits(splits):
+def test_caller_rows_give_the_same_bits(splits, impl):
+    """Also for the staged path, whose Q.K^T then reads the caller's rows for
+    the keys' latent dims (the pass still stages k_rope and q_lat)."""
     case = datagen.make_case("lc", **datagen.KIMI, prefix_len=[2300], parents=[datagen.random_tree(13, np.random.default_rng(5))],
                              seed=62, paged=True)
-    own = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC, num_splits=splits).run()
+    own = kdv.DeviceCase(case, impl=impl, num_splits=splits).run()
     o1, l1 = own.results()
-    mirror = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC, num_splits=splits)
+    mirror = kdv.DeviceCase(case, impl=impl, num_splits=splits)
     v16 = torch.empty(2300 + 13, 512, dtype=torch.float16, device="cuda")
     kdv.kdv_latent_f16(mirror.params, v16)
     mirror.params.v16 = v16.data_ptr()
