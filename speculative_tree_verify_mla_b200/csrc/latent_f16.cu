@@ -23,10 +23,11 @@
 // input below 2^-14 in magnitude was rounded to an fp16 subnormal), their
 // rope dims from the staged rows.
 //
-// HBM-bound: 1 KB read and 1 KB written per key (+128 B read and written
-// when staging). One warp per key row, lane l owning dims [16 l, 16 l + 16)
-// (and, for lanes 0-7, k_rope bytes [16 l, 16 l + 16)); each warp keeps four
-// rows' loads in flight.
+// HBM-bound: 1 KB read and 1 KB written per key; staging adds 128 B read and
+// written per key (k_rope) and 1 KB read and written per query row (q_lat).
+// One warp per key row, lane l owning dims [16 l, 16 l + 16) (and, for lanes
+// 0-7, k_rope bytes [16 l, 16 l + 16)); each warp keeps four rows' loads in
+// flight. The query rows follow, one warp per row over the whole grid.
 #include <cuda_fp16.h>
 
 #include "kdv_internal.cuh"
