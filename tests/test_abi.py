@@ -315,6 +315,15 @@ def test_staged_workspace_size(lib):
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC_STAGED,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
     assert kdv.kdv_verify_attn_workspace(p) == al(103 * 1024) + 256 + al(103 * 64 * 2) + 3 * 4 * 512 * 2
+    # the caller's fp16 rows: the staged region starts the workspace ...
+    p.v16 = 0x10000
+    assert kdv.kdv_verify_attn_workspace(p) == 256 + al(103 * 64 * 2) + 3 * 4 * 512 * 2
+    # ... or follows the merge region (3 splits: 3 * 12 partial rows)
+    p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC_STAGED,
+                page_table=0x7000, num_splits=3, h_prefix_len=[100], h_tree_T=[3], v16=0x10000)
+    parts = 3 * 3 * 4
+    assert kdv.kdv_verify_attn_workspace(p) == \
+        al(al(parts * 512 * 2) + parts * 4) + 256 + al(103 * 64 * 2) + 3 * 4 * 512 * 2
     # reading the pool through the page table needs only the fp16 rows
     p = _params(dtype=kdv.KDV_BF16, d_latent=512, d_rope=64, impl=kdv.KDV_IMPL_TC,
                 page_table=0x7000, num_splits=1, h_prefix_len=[100], h_tree_T=[3])
