@@ -1,6 +1,7 @@
 """GPU parity of the tensor-core (tcgen05/TMEM/TMA) verify kernel vs the oracle,
 through the C ABI. Kimi/DeepSeekV3 latent dims (512 + 64), bf16 inputs, the
 2-SM-MMA kernel on 4-CTA clusters."""
+import dataclasses
 import math
 
 import numpy as np
@@ -178,6 +179,20 @@ def test_tc_staged_bad_slot_reported():
     dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_STAGED, num_splits=0).run()
     dc.results()
     assert dc.error_flag() == kdv.KDV_DERR_BAD_SLOT
+
+
+@pytest.mark.parametrize("value,err", [(-65536.0, kdv.KDV_DERR_RANGE), (65280.0, 0)])
+def test_tc_staged_q_lat_range(value, err):
+    """The staged path reads q_lat in fp16: a value fp16 cannot hold is
+    reported; the largest bf16 magnitude below it is accepted."""
+    case = datagen.make_case("sq", **datagen.KIMI, prefix_len=[300], parents=[datagen.chain_tree(5)],
+                             seed=4, paged=True)
+    q = case.q.copy()
+    q[7, 100] = value
+    case = dataclasses.replace(case, q=q)
+    dc = kdv.DeviceCase(case, impl=kdv.KDV_IMPL_TC_STAGED, num_splits=0).run()
+    dc.results()
+    assert dc.error_flag() == err
 
 
 def test_tc_staged_without_page_table_is_tc():
